@@ -1,0 +1,341 @@
+"""Benchmark of one hot-path step: corrected attention of the current chunk over the packed
+INT2 cache plus the unquantised chunk, then quantise-append of the finished chunk.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). `value` is attention TFLOP/s of the whole job (algorithmic
+4*d FLOPs per (query, visible key) pair) over the device-timed steps, max over ranks. Inputs are
+resident in HBM; L2 is flushed (a 256 MiB write) between timed steps, outside the timed events.
+`--impl reference` times the CPU oracle instead (bounded samples of the same workload).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_kv_cache_19_b200 import api  # noqa: E402
+from quantized_kv_cache_19_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "corrected INT2-KV attention TFLOP/s & packed-cache GB/s, % of B200 roofline"
+DEFAULT_WORKLOAD = "bf16_int2"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def describe(w) -> str:
+    return (f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} d{w.d} Lq{w.Lq} Lcur{w.Lcur} Lc{w.Lc} "
+            f"INT{w.bits} G{w.group} meta {w.meta} {w.dtype}{' causal' if w.causal else ''}")
+
+
+# ------------------------------------------------------------------------------------ ranks
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a float over ranks (the slowest rank's time decides a multi-GPU number)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h))
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "samples": len(self.samples),
+                "reasons": [n for bit, n in self.REASONS.items() if self.reasons & bit]}
+
+
+# ------------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, x_cpu, budget_s: float, seed: int = 0):
+    """Oracle on a bounded sample of one step: quantise the whole current chunk, then corrected
+    attention of n query rows per KV head over the full cache. Returns (seconds, flops, sample text)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    scale = 1.0 / math.sqrt(w.d)
+    K = {k: v.float().numpy() for k, v in x_cpu.items()}
+    t0 = time.perf_counter()
+    oracle.build_cache(K["K_cur"], K["V_cur"], w.bits, w.group, w.meta)      # the step's append
+    t_quant = time.perf_counter() - t0
+    cache = oracle.build_cache(K["K_src"], K["V_src"], w.bits, w.group, w.meta)   # state, untimed
+    rng = np.random.default_rng(seed)
+    total_rows = (w.Hq // w.Hkv) * w.Lq
+    n = 16
+    spent, flops_done, rows_done = 0.0, 0.0, 0
+    while True:
+        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+        t0 = time.perf_counter()
+        oracle.corrected_attention(K["Q"], cache, K["K_cur"], K["V_cur"], correct=1, causal=w.causal,
+                                   scale=scale, rows=rows)
+        dt = time.perf_counter() - t0
+        spent += dt
+        rows_done += len(rows) * w.B * w.Hkv
+        flops_done += 4.0 * w.d * len(rows) * w.B * w.Hkv * (w.Lc + w.Lcur)
+        if spent >= budget_s or len(rows) == total_rows:
+            break
+        n = min(total_rows, n * 2)
+    blas = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
+    cores = blas or os.cpu_count()
+    all_rows = total_rows * w.B * w.Hkv
+    est_s = t_quant + spent * all_rows / rows_done           # linear in query rows
+    full_flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
+    text = (f"oracle (numpy fp64 attention, fp32 quantiser): quantise-append of the whole {w.Lcur}-token "
+            f"chunk ({t_quant:.2f} s) + corrected attention of {rows_done} of {all_rows} query rows "
+            f"({spent:.2f} s); full step extrapolated linearly in rows to {est_s:.1f} s")
+    return est_s, full_flops, text, cores
+
+
+# ------------------------------------------------------------------------------------ GPU arm
+def run_ours(args, world, rank, local):
+    w = WORKLOADS[args.workload]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_kind = load_peaks()
+    api.load_library()
+
+    x = make_inputs(w, device="cuda", seed=w.seed + rank)      # each rank: its own problem (weak scaling)
+    cap = api.round_capacity(w.Lc + w.Lcur)
+    cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, cap, w.meta, device=dev)
+    for t0 in range(0, w.Lc, max(w.Lcur, 1)):                   # previous chunks, appended one by one
+        t1 = min(w.Lc, t0 + max(w.Lcur, 1))
+        api.kv_quantize_append(cache, x["K_src"][:, :, t0:t1].contiguous(), x["V_src"][:, :, t0:t1].contiguous())
+    O = torch.empty_like(x["Q"])
+    LSE = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        cache.length = w.Lc
+        api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1, causal=w.causal, out=O, lse=LSE)
+        api.kv_quantize_append(cache, x["K_cur"], x["V_cur"])
+
+    for _ in range(args.warmup):
+        step()
+        flush.fill_(1)
+    torch.cuda.synchronize()
+    assert api.device_status() == 0
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            cache.length = w.Lc
+            ev[i][0].record(stream)
+            api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1, causal=w.causal,
+                                    out=O, lse=LSE)
+            ev[i][1].record(stream)
+            api.kv_quantize_append(cache, x["K_cur"], x["V_cur"])
+            ev[i][2].record(stream)
+            flush.fill_(i & 0xFF)
+        torch.cuda.synchronize()
+    barrier(world)
+    attn_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    qa_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [a + q for a, q in zip(attn_ms, qa_ms)]
+    status = api.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed steps")
+
+    # end to end through the public API with host buffers: H2D of the step's inputs, D2H of O, LSE
+    pin = {k: x[k].cpu().pin_memory() for k in ("Q", "K_cur", "V_cur")}
+    dev_in = {k: torch.empty_like(x[k]) for k in pin}
+    O_host = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    L_host = torch.empty(LSE.shape, dtype=LSE.dtype).pin_memory()
+    n_e2e = min(K, 50)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
+    for i in range(n_e2e + 3):
+        flush.fill_(i & 0xFF)
+        if i >= 3:
+            e2e_ev[i - 3][0].record(stream)
+        for k in pin:
+            dev_in[k].copy_(pin[k], non_blocking=True)
+        cache.length = w.Lc
+        api.corrected_attention(dev_in["Q"], cache, dev_in["K_cur"], dev_in["V_cur"], correct=1,
+                                causal=w.causal, out=O, lse=LSE)
+        api.kv_quantize_append(cache, dev_in["K_cur"], dev_in["V_cur"])
+        O_host.copy_(O, non_blocking=True)
+        L_host.copy_(LSE, non_blocking=True)
+        if i >= 3:
+            e2e_ev[i - 3][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in e2e_ev)
+
+    flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
+    mean_step = statistics.mean(step_ms)
+    mean_attn = statistics.mean(attn_ms)
+    mean_qa = statistics.mean(qa_ms)
+    ms_step = reduce_max(mean_step, world, dev)
+    ms_attn = reduce_max(mean_attn, world, dev)
+    ms_e2e = reduce_max(e2e_ms, world, dev)
+    packed = cache.packed_bytes(w.Lc)
+    esz = x["K_cur"].element_size()
+    qa_bytes = w.B * w.Hkv * w.Lcur * (2 * w.d * esz + 2 * (w.d * w.bits // 8) + 2 * w.n_groups * 2 *
+                                        (2 if w.meta == "f16" else 4))
+    peak_t = float(peaks["bf16_tflops"])
+    achieved = flops / (ms_attn * 1e-3) / 1e12
+    result = {
+        "metric": METRIC,
+        "value": round(world * flops / (ms_step * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(w), "step": "corrected attention (correct=1) + quantise-append of the chunk",
+                   "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "packed_cache_gbs": round(packed / (ms_attn * 1e-3) / 1e9, 1),
+        "roofline": {"bound": "tensor", "kernel": "corrected_attention_kernel",
+                     "achieved": round(achieved, 2), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_t, 4), "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                     "traffic": args.traffic, "ms_per_launch": round(ms_attn, 5),
+                     "flops_per_launch": flops},
+        "quant_append": {"bound": "hbm", "ms_per_launch": round(mean_qa, 5),
+                         "bytes_per_launch": qa_bytes,
+                         "achieved_gbs": round(qa_bytes / (mean_qa * 1e-3) / 1e9, 1),
+                         "peak_gbs": float(peaks["hbm_gbs"]),
+                         "frac": round(qa_bytes / (mean_qa * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)},
+        "e2e": {"value": round(world * flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(ms_e2e, 5),
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
+                "d2h_bytes_per_step": O.numel() * O.element_size() + LSE.numel() * LSE.element_size()},
+        "gpu_launches": 2 * K,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        x_cpu = make_inputs(w, device="cpu")
+        est_s, full_flops, text, cores = oracle_sample(w, x_cpu, args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(full_flops / est_s / 1e12, 6), "unit": "TFLOP/s",
+                                  "cores": cores, "kind": "oracle", "sample": text}
+    return result
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on bounded samples of the same workload."""
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    x_cpu = make_inputs(w, device="cpu")
+    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    times, text, cores = [], "", os.cpu_count()
+    for i in range(args.warmup + args.steps):
+        est_s, full_flops, text, cores = oracle_sample(w, x_cpu, per_step, seed=i)
+        if i >= args.warmup:
+            times.append(est_s)
+    mean_s = statistics.mean(times)
+    value = full_flops / mean_s / 1e12
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(mean_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(w), "step": "corrected attention (correct=1) + quantise-append of the chunk"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {text}"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of the current kernel")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_ours(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,148 @@
+/*
+ * qkv.h — C ABI of libqkv: a low-bit (INT2/INT4) group-quantised KV cache and
+ * Jensen-bias-corrected chunk-wise attention over it, for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Quantized Keys Steal Attention: Bias Correction for KV-Cache Compression
+ * in Video Diffusion" (Tuncer, Becker, Pfeil), as summarised on agents-report.net
+ * ("KV-Cache 量化導致的 Jensen 偏差：以每分數校正恢復影片擴散品質") and in the abstract on
+ * fugumt.com. The current chunk's queries attend over the quantised cache of the previous
+ * chunks plus the unquantised current chunk; every cached-key score has the correction
+ * b = (1/(24 d)) sum_c q_c^2 Delta_c^2 subtracted before the softmax (summary, section 方法).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, 16-byte aligned, contiguous
+ *    row-major. The library never allocates, frees or synchronises: work is enqueued on the
+ *    caller's CUDA stream (`stream` is a cudaStream_t; NULL means the legacy default stream).
+ *  - Arguments are validated on the host before anything is enqueued. A rejected call returns
+ *    QKV_ERR_INVALID_ARG, QKV_ERR_UNSUPPORTED or QKV_ERR_CAPACITY and changes nothing.
+ *  - A launch failure returns QKV_ERR_CUDA. qkv_last_error() gives a message (per host thread).
+ *  - Kernels bound every internal wait. A wait that runs out sets a word in device memory and
+ *    the kernel returns early; qkv_device_status() reads that word (it synchronises the device).
+ *  - There is no CPU fallback and no other backend: every combination that is not compiled
+ *    returns QKV_ERR_UNSUPPORTED.
+ *  - Calls that touch the same cache must be ordered by the caller (e.g. one stream).
+ */
+#ifndef QKV_H
+#define QKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QKV_ABI_VERSION 1
+/* Tokens per cache tile; a cache's capacity must be a multiple of it. */
+#define QKV_CACHE_TILE 128
+
+typedef enum {
+  QKV_OK = 0,
+  QKV_ERR_INVALID_ARG = -1, /* null/misaligned pointer, bad size or shape */
+  QKV_ERR_UNSUPPORTED = -2, /* valid request that no compiled kernel serves */
+  QKV_ERR_CAPACITY = -3,    /* append would exceed the cache capacity */
+  QKV_ERR_CUDA = -4,        /* CUDA runtime or launch error */
+  QKV_ERR_TIMEOUT = -5      /* a kernel's bounded wait ran out (from qkv_device_status) */
+} qkv_status;
+
+typedef enum { QKV_F32 = 0, QKV_BF16 = 1, QKV_F16 = 2 } qkv_dtype;
+
+/*
+ * Packed KV cache (plain descriptor; the caller owns all four buffers).
+ *
+ * Quantiser (summary, section 問題 "INT4/INT2 integer quantisation"; abstract "quantisation step
+ * sizes"): for each (batch b, KV head h, token t) and each group g of `group` consecutive
+ * channels, asymmetric min-max: step = (max - min) / (2^bits - 1) and zero-point = min, both in
+ * IEEE fp32, then stored in `meta_dtype` (round to nearest even). Codes are taken against the
+ * STORED values: code = clamp(rint((x - zp) * (1/step)), 0, 2^bits - 1), each operation one
+ * correctly rounded fp32 operation, ties to even; a zero step gives code 0.
+ *
+ *  k_codes, v_codes : uint8 [B][H_kv][capacity][d*bits/8]; channel c of a token at bit c*bits of
+ *                     the row's little-endian bit string (byte c*bits/8, bit c*bits%8).
+ *  k_meta, v_meta   : meta_dtype [B][H_kv][capacity][d/group][2]; element 0 = step, 1 = zero-point.
+ *  length           : tokens currently held per (b, h) (positions 0..length-1 are valid).
+ *  capacity         : tokens the buffers hold per (b, h); a positive multiple of QKV_CACHE_TILE.
+ * Supported: d in {64, 128}; bits in {2, 4}; group in {32, 64, 128} dividing d;
+ * meta_dtype in {QKV_F32, QKV_F16}.
+ */
+typedef struct {
+  int32_t B, H_kv, d, bits, group;
+  int32_t meta_dtype;
+  int64_t capacity;
+  int64_t length;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  void* k_meta;
+  void* v_meta;
+} qkv_cache;
+
+/* Bytes of ONE codes buffer and of ONE meta buffer for the given cache shape (host only). */
+qkv_status qkv_cache_bytes(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int32_t group,
+                           int32_t meta_dtype, int64_t capacity, size_t* codes_bytes_each,
+                           size_t* meta_bytes_each);
+
+/*
+ * Quantise a finished chunk and append it to the cache (QuantWM page on pchao.org, 方法概览:
+ * each cache block is quantised once, after it is built).
+ *  K, V     : in_dtype [B][H_kv][L_new][d] (QKV_F32 or QKV_BF16), device, 16-byte aligned.
+ *  L_new    : tokens to append, >= 0 (0 is a no-op).
+ * Writes codes and (step, zero-point) for positions length .. length+L_new-1 and, once the
+ * kernel is enqueued, advances cache->length by L_new. Returns QKV_ERR_CAPACITY (and enqueues
+ * nothing) if length + L_new > capacity.
+ */
+qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const void* V, int32_t in_dtype,
+                              int64_t L_new, void* stream);
+
+/* Device workspace that corrected_attention needs for this shape (may be 0). */
+qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H_q, int64_t L_q,
+                                               int64_t L_cur, size_t* bytes);
+
+/*
+ * Corrected chunk attention (summary, sections 方法 and 為何校正有效; scores q.k*scale as in the
+ * QuantWM page, eq. (5)). For each query row, one softmax runs over the cache's first
+ * cache->length keys followed by the L_cur current keys. Cached-key scores have the Jensen
+ * correction subtracted when correct = 1:
+ *     b_j = (scale^2 / 24) * sum_c q_c^2 * step_{j, c/group}^2   (= (1/(24 d)) ... at scale 1/sqrt(d)).
+ *  Q            : dtype [B][H_q][L_q][d]; dtype QKV_F32 or QKV_BF16. H_q % H_kv == 0; query head
+ *                 hq reads KV head hq / (H_q / H_kv).
+ *  K_cur, V_cur : dtype [B][H_kv][L_cur][d], the unquantised current chunk (may be NULL if L_cur=0).
+ *  correct      : 0 = plain attention over the dequantised cache, 1 = Taylor correction.
+ *  causal_cur   : 1 = query i sees current key j only if j <= i + (L_cur - L_q); the cache is
+ *                 always fully visible.
+ *  scale        : score scale; <= 0 means 1/sqrt(d).
+ *  O            : dtype [B][H_q][L_q][d] (same type as Q). LSE: fp32 [B][H_q][L_q], natural log
+ *                 of the row's softmax denominator (-inf and O = 0 for a row that sees no key).
+ *  workspace    : device scratch of at least corrected_attention_workspace_bytes() (may be NULL
+ *                 when that is 0).
+ * L_cur = 0 and cache->length = 0 together are rejected (no keys at all).
+ */
+qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                               const qkv_cache* cache, const void* K_cur, const void* V_cur,
+                               int64_t L_cur, int32_t correct, int32_t causal_cur, float scale,
+                               void* O, float* LSE, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * The correction term alone, for checking: bias fp32 [B][H_q][L_q][cache->length] with
+ * bias[b][hq][i][j] = (scale^2/24) * sum_c Q[b][hq][i][c]^2 * step_{j, c/group}^2, computed by
+ * the same device functions corrected_attention uses (fp32).
+ */
+qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                           const qkv_cache* cache, float scale, float* bias, void* stream);
+
+/*
+ * Reads the library's device status word (0 = no error, else a qkv_status such as
+ * QKV_ERR_TIMEOUT) into *code; clears it when reset != 0. Synchronises the current device.
+ */
+qkv_status qkv_device_status(int32_t reset, int32_t* code);
+
+const char* qkv_status_string(int32_t status);
+/* Message of the last failed call on this host thread ("" if none). */
+const char* qkv_last_error(void);
+int32_t qkv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKV_H */

@@ -1,0 +1,258 @@
+// C ABI of libqkv: argument validation, dispatch to the kernels, error reporting.
+// The declarations, layouts and error behaviour are documented in include/qkv.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/qkv.h"
+#include "qkv_internal.h"
+
+#define QKV_API extern "C" __attribute__((visibility("default")))
+
+namespace qkv {
+
+// Device status word of this library: 0 = ok, else a negative qkv_status set by a kernel.
+__device__ int g_device_status;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+qkv_status fail(qkv_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+qkv_status fail(qkv_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+qkv_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(QKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Address of g_device_status on the current device (looked up once per device).
+int* status_word(cudaError_t* err) {
+  static int* addr[64] = {nullptr};
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, g_device_status);
+    if (*err != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
+qkv_status check_shape(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int32_t group,
+                       int32_t meta_dtype, int64_t capacity) {
+  if (B < 1 || H_kv < 1) return fail(QKV_ERR_INVALID_ARG, "B and H_kv must be >= 1");
+  if (capacity < QKV_CACHE_TILE || capacity % QKV_CACHE_TILE)
+    return fail(QKV_ERR_INVALID_ARG, "capacity must be a positive multiple of %d", QKV_CACHE_TILE);
+  if (d != 64 && d != 128) return fail(QKV_ERR_UNSUPPORTED, "head dim %d not supported (64, 128)", d);
+  if (bits != 2 && bits != 4) return fail(QKV_ERR_UNSUPPORTED, "bits %d not supported (2, 4)", bits);
+  if (group != 32 && group != 64 && group != 128)
+    return fail(QKV_ERR_UNSUPPORTED, "group %d not supported (32, 64, 128)", group);
+  if (d % group) return fail(QKV_ERR_INVALID_ARG, "group %d does not divide d %d", group, d);
+  if (meta_dtype != QKV_F32 && meta_dtype != QKV_F16)
+    return fail(QKV_ERR_UNSUPPORTED, "meta dtype must be QKV_F32 or QKV_F16");
+  return QKV_OK;
+}
+
+qkv_status check_cache(const qkv_cache* c) {
+  if (c == nullptr) return fail(QKV_ERR_INVALID_ARG, "cache is NULL");
+  qkv_status s = check_shape(c->B, c->H_kv, c->d, c->bits, c->group, c->meta_dtype, c->capacity);
+  if (s != QKV_OK) return s;
+  if (c->length < 0 || c->length > c->capacity)
+    return fail(QKV_ERR_INVALID_ARG, "cache length %lld outside [0, capacity]",
+                static_cast<long long>(c->length));
+  if (!c->k_codes || !c->v_codes || !c->k_meta || !c->v_meta)
+    return fail(QKV_ERR_INVALID_ARG, "cache buffer is NULL");
+  if (!aligned16(c->k_codes) || !aligned16(c->v_codes) || !aligned16(c->k_meta) ||
+      !aligned16(c->v_meta))
+    return fail(QKV_ERR_INVALID_ARG, "cache buffers must be 16-byte aligned");
+  return QKV_OK;
+}
+
+bool in_dtype_ok(int32_t dt) { return dt == QKV_F32 || dt == QKV_BF16; }
+
+}  // namespace
+}  // namespace qkv
+
+using namespace qkv;
+
+QKV_API int32_t qkv_abi_version(void) { return QKV_ABI_VERSION; }
+
+QKV_API const char* qkv_status_string(int32_t s) {
+  switch (s) {
+    case QKV_OK: return "ok";
+    case QKV_ERR_INVALID_ARG: return "invalid argument";
+    case QKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QKV_ERR_CAPACITY: return "cache capacity exceeded";
+    case QKV_ERR_CUDA: return "CUDA error";
+    case QKV_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+QKV_API const char* qkv_last_error(void) { return t_last_error.c_str(); }
+
+QKV_API qkv_status qkv_cache_bytes(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int32_t group,
+                                   int32_t meta_dtype, int64_t capacity, size_t* codes_bytes_each,
+                                   size_t* meta_bytes_each) {
+  t_last_error.clear();
+  qkv_status s = check_shape(B, H_kv, d, bits, group, meta_dtype, capacity);
+  if (s != QKV_OK) return s;
+  if (!codes_bytes_each || !meta_bytes_each) return fail(QKV_ERR_INVALID_ARG, "NULL output");
+  const size_t tokens = static_cast<size_t>(B) * H_kv * static_cast<size_t>(capacity);
+  *codes_bytes_each = tokens * (d * bits / 8);
+  *meta_bytes_each = tokens * (d / group) * 2 * (meta_dtype == QKV_F16 ? 2 : 4);
+  return QKV_OK;
+}
+
+QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const void* V,
+                                      int32_t in_dtype, int64_t L_new, void* stream) {
+  t_last_error.clear();
+  qkv_status s = check_cache(cache);
+  if (s != QKV_OK) return s;
+  if (!in_dtype_ok(in_dtype)) return fail(QKV_ERR_UNSUPPORTED, "input dtype must be F32 or BF16");
+  if (L_new < 0) return fail(QKV_ERR_INVALID_ARG, "L_new must be >= 0");
+  if (L_new > cache->capacity - cache->length)
+    return fail(QKV_ERR_CAPACITY, "append of %lld tokens to a cache holding %lld of %lld",
+                static_cast<long long>(L_new), static_cast<long long>(cache->length),
+                static_cast<long long>(cache->capacity));
+  if (L_new == 0) return QKV_OK;
+  if (!K || !V) return fail(QKV_ERR_INVALID_ARG, "K or V is NULL");
+  if (!aligned16(K) || !aligned16(V)) return fail(QKV_ERR_INVALID_ARG, "K and V must be 16-byte aligned");
+  QuantAppendParams p;
+  p.K = K; p.V = V;
+  p.k_codes = cache->k_codes; p.v_codes = cache->v_codes;
+  p.k_meta = cache->k_meta; p.v_meta = cache->v_meta;
+  p.rows = static_cast<int64_t>(cache->B) * cache->H_kv * L_new;
+  p.L_new = L_new;
+  p.capacity = cache->capacity;
+  p.start = cache->length;
+  p.d = cache->d;
+  p.group = cache->group;
+  cudaError_t e = launch_quantize_append(p, in_dtype, cache->meta_dtype, cache->bits,
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_quantize_append launch");
+  cache->length += L_new;
+  return QKV_OK;
+}
+
+QKV_API qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H_q,
+                                                       int64_t L_q, int64_t L_cur, size_t* bytes) {
+  t_last_error.clear();
+  qkv_status s = check_cache(cache);
+  if (s != QKV_OK) return s;
+  if (!bytes) return fail(QKV_ERR_INVALID_ARG, "NULL output");
+  if (H_q < 1 || H_q % cache->H_kv || L_q < 0 || L_cur < 0)
+    return fail(QKV_ERR_INVALID_ARG, "bad H_q / L_q / L_cur");
+  *bytes = 0;
+  return QKV_OK;
+}
+
+QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                                       const qkv_cache* cache, const void* K_cur,
+                                       const void* V_cur, int64_t L_cur, int32_t correct,
+                                       int32_t causal_cur, float scale, void* O, float* LSE,
+                                       void* workspace, size_t workspace_bytes, void* stream) {
+  t_last_error.clear();
+  (void)workspace;
+  (void)workspace_bytes;
+  qkv_status s = check_cache(cache);
+  if (s != QKV_OK) return s;
+  if (!in_dtype_ok(dtype)) return fail(QKV_ERR_UNSUPPORTED, "dtype must be F32 or BF16");
+  if (H_q < 1 || H_q % cache->H_kv)
+    return fail(QKV_ERR_INVALID_ARG, "H_q %d must be a positive multiple of H_kv %d", H_q,
+                cache->H_kv);
+  if (L_q < 0 || L_cur < 0) return fail(QKV_ERR_INVALID_ARG, "negative length");
+  if (correct != 0 && correct != 1) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0 or 1");
+  if (causal_cur != 0 && causal_cur != 1) return fail(QKV_ERR_INVALID_ARG, "causal_cur must be 0 or 1");
+  if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
+  if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
+  if (L_q == 0) return QKV_OK;
+  if (!Q || !O || !LSE) return fail(QKV_ERR_INVALID_ARG, "Q, O or LSE is NULL");
+  if (L_cur > 0 && (!K_cur || !V_cur)) return fail(QKV_ERR_INVALID_ARG, "K_cur or V_cur is NULL");
+  if (!aligned16(Q) || !aligned16(O) || !aligned16(LSE) || (L_cur > 0 && (!aligned16(K_cur) || !aligned16(V_cur))))
+    return fail(QKV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(H_q / cache->H_kv) * L_q;
+  if ((rows + 127) / 128 > 2147483647LL || static_cast<int64_t>(cache->B) * cache->H_kv > 65535)
+    return fail(QKV_ERR_UNSUPPORTED, "grid too large");
+  cudaError_t e;
+  int* status = status_word(&e);
+  if (!status) return cuda_fail(e, "device status word");
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(cache->d));
+  const float log2e = 1.4426950408889634f;
+  AttnParams p;
+  p.Q = Q; p.K_cur = K_cur; p.V_cur = V_cur; p.O = O; p.LSE = LSE;
+  p.k_codes = cache->k_codes; p.v_codes = cache->v_codes;
+  p.k_meta = cache->k_meta; p.v_meta = cache->v_meta;
+  p.status = status;
+  p.Lq = L_q; p.Lc = cache->length; p.Lcur = L_cur; p.capacity = cache->capacity;
+  p.B = cache->B; p.Hq = H_q; p.Hkv = cache->H_kv; p.r = H_q / cache->H_kv;
+  p.group = cache->group; p.n_groups = cache->d / cache->group;
+  p.correct = correct; p.causal = causal_cur;
+  p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
+  p.scale_log2 = sc * log2e;
+  p.wcoef_log2 = sc * sc / 24.0f * log2e;
+  e = launch_attention(p, cache->d, cache->bits, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");
+  return QKV_OK;
+}
+
+QKV_API qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                                   const qkv_cache* cache, float scale, float* bias, void* stream) {
+  t_last_error.clear();
+  qkv_status s = check_cache(cache);
+  if (s != QKV_OK) return s;
+  if (!in_dtype_ok(dtype)) return fail(QKV_ERR_UNSUPPORTED, "dtype must be F32 or BF16");
+  if (H_q < 1 || H_q % cache->H_kv) return fail(QKV_ERR_INVALID_ARG, "bad H_q");
+  if (L_q < 0) return fail(QKV_ERR_INVALID_ARG, "negative L_q");
+  if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
+  if (L_q == 0 || cache->length == 0) return QKV_OK;
+  if (!Q || !bias) return fail(QKV_ERR_INVALID_ARG, "Q or bias is NULL");
+  if (!aligned16(Q) || !aligned16(bias)) return fail(QKV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if ((cache->length + 255) / 256 > 65535 ||
+      static_cast<int64_t>(cache->B) * H_q * L_q > 2147483647LL)
+    return fail(QKV_ERR_UNSUPPORTED, "bias grid too large");
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(cache->d));
+  BiasParams p;
+  p.Q = Q; p.k_meta = cache->k_meta; p.bias = bias;
+  p.Lq = L_q; p.Lc = cache->length; p.capacity = cache->capacity;
+  p.B = cache->B; p.Hq = H_q; p.Hkv = cache->H_kv; p.r = H_q / cache->H_kv;
+  p.d = cache->d; p.group = cache->group; p.n_groups = cache->d / cache->group;
+  p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
+  p.wcoef = sc * sc / 24.0f;
+  cudaError_t e = launch_jensen_bias(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "qkv_jensen_bias launch");
+  return QKV_OK;
+}
+
+QKV_API qkv_status qkv_device_status(int32_t reset, int32_t* code) {
+  t_last_error.clear();
+  if (!code) return fail(QKV_ERR_INVALID_ARG, "NULL output");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "synchronise");
+  int* addr = status_word(&e);
+  if (!addr) return cuda_fail(e, "device status word");
+  int v = 0;
+  e = cudaMemcpy(&v, addr, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  if (reset && v != 0) {
+    const int zero = 0;
+    e = cudaMemcpy(addr, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "reset device status");
+  }
+  *code = v;
+  return QKV_OK;
+}

@@ -1,0 +1,65 @@
+// Host-side declarations shared by the translation units of libqkv (not part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qkv {
+
+enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
+
+// Quantise-and-append: K and V [B][H_kv][L_new][d] into the cache at positions start..start+L_new-1.
+struct QuantAppendParams {
+  const void* K;
+  const void* V;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  void* k_meta;
+  void* v_meta;
+  int64_t rows;      // B * H_kv * L_new token-head rows per tensor
+  int64_t L_new;
+  int64_t capacity;
+  int64_t start;
+  int d, group;
+};
+cudaError_t launch_quantize_append(const QuantAppendParams& p, int in_dtype, int meta_dtype,
+                                   int bits, cudaStream_t stream);
+
+// Corrected attention: one CTA per (128 packed query rows, batch * KV head).
+struct AttnParams {
+  const void* Q;
+  const void* K_cur;
+  const void* V_cur;
+  void* O;
+  float* LSE;
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const void* k_meta;
+  const void* v_meta;
+  int* status;
+  int64_t Lq, Lc, Lcur, capacity;
+  int B, Hq, Hkv, r;
+  int group, n_groups;
+  int correct, causal;
+  int in_f32, meta_f16;
+  float scale_log2;   // score scale * log2(e)
+  float wcoef_log2;   // scale^2 / 24 * log2(e): Jensen-correction coefficient in log2 units
+};
+size_t attention_smem_bytes(int d, int bits, int n_groups, int meta_bytes);
+cudaError_t launch_attention(const AttnParams& p, int d, int bits, cudaStream_t stream);
+
+// Jensen-correction term alone: bias[B][Hq][Lq][Lc] (natural units).
+struct BiasParams {
+  const void* Q;
+  const void* k_meta;
+  float* bias;
+  int64_t Lq, Lc, capacity;
+  int B, Hq, Hkv, r;
+  int d, group, n_groups;
+  int in_f32, meta_f16;
+  float wcoef;        // scale^2 / 24
+};
+cudaError_t launch_jensen_bias(const BiasParams& p, cudaStream_t stream);
+
+}  // namespace qkv

@@ -1,0 +1,97 @@
+"""The C-ABI library loads without a GPU, exports what include/qkv.h declares, and rejects bad
+arguments on the host (no CUDA call is made on any path exercised here)."""
+import ctypes
+
+import pytest
+
+from quantized_kv_cache_19_b200 import api
+
+
+def test_exports_every_header_function(lib):
+    names = api.header_functions()
+    assert {"kv_quantize_append", "corrected_attention", "qkv_jensen_bias", "qkv_cache_bytes",
+            "corrected_attention_workspace_bytes", "qkv_device_status", "qkv_status_string",
+            "qkv_last_error", "qkv_abi_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.qkv_abi_version() == 1
+
+
+def test_status_strings(lib):
+    assert lib.qkv_status_string(0) == b"ok"
+    assert lib.qkv_status_string(-3) == b"cache capacity exceeded"
+    assert lib.qkv_status_string(-5) == b"device wait timed out"
+
+
+@pytest.mark.parametrize("args,codes,meta", [
+    ((1, 2, 64, 2, 32, api.QKV_F32, 256), 2 * 256 * 16, 2 * 256 * 2 * 2 * 4),
+    ((1, 16, 128, 4, 64, api.QKV_F32, 5120), 16 * 5120 * 64, 16 * 5120 * 2 * 2 * 4),
+    ((1, 40, 128, 2, 128, api.QKV_F16, 99840), 40 * 99840 * 32, 40 * 99840 * 1 * 2 * 2),
+    ((4, 8, 128, 2, 64, api.QKV_F32, 131072), 32 * 131072 * 32, 32 * 131072 * 2 * 2 * 4),
+])
+def test_cache_bytes(lib, args, codes, meta):
+    cb, mb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.qkv_cache_bytes(*args, ctypes.byref(cb), ctypes.byref(mb)) == 0
+    assert (cb.value, mb.value) == (codes, meta)
+
+
+@pytest.mark.parametrize("args,status", [
+    ((1, 2, 64, 3, 32, api.QKV_F32, 256), api.QKV_ERR_UNSUPPORTED),     # 3-bit codes
+    ((1, 2, 96, 2, 32, api.QKV_F32, 256), api.QKV_ERR_UNSUPPORTED),     # head dim
+    ((1, 2, 64, 2, 128, api.QKV_F32, 256), api.QKV_ERR_INVALID_ARG),    # group > d
+    ((1, 2, 64, 2, 32, api.QKV_F32, 200), api.QKV_ERR_INVALID_ARG),     # capacity not a tile multiple
+    ((0, 2, 64, 2, 32, api.QKV_F32, 256), api.QKV_ERR_INVALID_ARG),
+    ((1, 2, 64, 2, 32, api.QKV_BF16, 256), api.QKV_ERR_UNSUPPORTED),    # meta must be f32 / f16
+])
+def test_cache_bytes_rejects(lib, args, status):
+    cb, mb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.qkv_cache_bytes(*args, ctypes.byref(cb), ctypes.byref(mb)) == status
+    assert lib.qkv_last_error() != b""
+
+
+def _fake_cache(**kw):
+    c = dict(B=1, H_kv=2, d=128, bits=2, group=64, meta_dtype=api.QKV_F32, capacity=256, length=0,
+             k_codes=0x10000, v_codes=0x20000, k_meta=0x30000, v_meta=0x40000)
+    c.update(kw)
+    return api.QkvCacheDesc(**c)
+
+
+def test_append_rejections(lib):
+    c = _fake_cache(length=200)
+    s = lib.kv_quantize_append(ctypes.byref(c), ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000),
+                               api.QKV_BF16, 57, None)
+    assert s == api.QKV_ERR_CAPACITY and c.length == 200
+    assert b"exceed" in lib.qkv_last_error() or b"append" in lib.qkv_last_error()
+    assert lib.kv_quantize_append(ctypes.byref(c), ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000),
+                                  api.QKV_F16, 8, None) == api.QKV_ERR_UNSUPPORTED
+    assert lib.kv_quantize_append(ctypes.byref(c), ctypes.c_void_p(0x50008), ctypes.c_void_p(0x60000),
+                                  api.QKV_BF16, 8, None) == api.QKV_ERR_INVALID_ARG
+    assert lib.kv_quantize_append(ctypes.byref(c), None, None, api.QKV_BF16, 0, None) == 0  # no-op
+    assert c.length == 200
+    bad = _fake_cache(k_meta=0x30004)
+    assert lib.kv_quantize_append(ctypes.byref(bad), ctypes.c_void_p(0x50000), ctypes.c_void_p(0x60000),
+                                  api.QKV_BF16, 8, None) == api.QKV_ERR_INVALID_ARG
+    assert lib.kv_quantize_append(None, None, None, api.QKV_BF16, 8, None) == api.QKV_ERR_INVALID_ARG
+
+
+def test_attention_rejections(lib):
+    c = _fake_cache(length=0)
+    P = ctypes.c_void_p
+    q, o, l = P(0x70000), P(0x80000), P(0x90000)
+    call = lambda **kw: lib.corrected_attention(
+        kw.get("Q", q), kw.get("dt", api.QKV_BF16), kw.get("Hq", 4), kw.get("Lq", 16), ctypes.byref(kw.get("c", c)),
+        kw.get("K", P(0xA0000)), kw.get("V", P(0xB0000)), kw.get("Lcur", 0), kw.get("corr", 1), 0,
+        kw.get("scale", 0.0), o, l, None, 0, None)
+    assert call() == api.QKV_ERR_INVALID_ARG                         # no keys at all
+    c2 = _fake_cache(length=100)
+    assert call(c=c2, Hq=3) == api.QKV_ERR_INVALID_ARG               # H_q not a multiple of H_kv
+    assert call(c=c2, dt=api.QKV_F16) == api.QKV_ERR_UNSUPPORTED
+    assert call(c=c2, corr=2) == api.QKV_ERR_UNSUPPORTED             # exact correction is oracle-only
+    assert call(c=c2, Q=P(0x70002)) == api.QKV_ERR_INVALID_ARG       # misaligned
+    assert call(c=c2, Lcur=8, K=None) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, scale=float("nan")) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, Lq=0) == 0                                     # empty query chunk: no-op
+    ws = ctypes.c_size_t(1)
+    assert lib.corrected_attention_workspace_bytes(ctypes.byref(c2), 4, 16, 8, ctypes.byref(ws)) == 0
+    assert lib.qkv_jensen_bias(q, api.QKV_BF16, 3, 16, ctypes.byref(c2), 0.0, P(0xC0000), None) == \
+        api.QKV_ERR_INVALID_ARG
