@@ -46,8 +46,9 @@ struct AttnParams {
   float scale_log2;   // score scale * log2(e)
   float wcoef_log2;   // scale^2 / 24 * log2(e): Jensen-correction coefficient in log2 units
 };
-size_t attention_smem_bytes(int d, int bits, int n_groups, int meta_bytes);
-cudaError_t launch_attention(const AttnParams& p, int d, int bits, cudaStream_t stream);
+// bf16 inputs: tcgen05 kernel. fp32 inputs: CUDA-core fp32 kernel.
+cudaError_t launch_attention_bf16(const AttnParams& p, int d, int bits, cudaStream_t stream);
+cudaError_t launch_attention_f32(const AttnParams& p, int d, int bits, cudaStream_t stream);
 
 // Jensen-correction term alone: bias[B][Hq][Lq][Lc] (natural units).
 struct BiasParams {
