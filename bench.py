@@ -134,20 +134,20 @@ def oracle_sample(w, x_cpu, budget_s: float, seed: int = 0):
     cache = oracle.build_cache(K["K_src"], K["V_src"], w.bits, w.group, w.meta)   # state, untimed
     rng = np.random.default_rng(seed)
     total_rows = (w.Hq // w.Hkv) * w.Lq
-    n = 16
-    spent, flops_done, rows_done = 0.0, 0.0, 0
-    while True:
-        rows = np.sort(rng.choice(total_rows, size=min(n, total_rows), replace=False))
+    order = rng.permutation(total_rows)            # rows drawn without replacement, in batches
+    n, start = 16, 0
+    spent, rows_done = 0.0, 0
+    while start < total_rows:
+        rows = np.sort(order[start:start + n])
         t0 = time.perf_counter()
         oracle.corrected_attention(K["Q"], cache, K["K_cur"], K["V_cur"], correct=1, causal=w.causal,
                                    scale=scale, rows=rows)
-        dt = time.perf_counter() - t0
-        spent += dt
+        spent += time.perf_counter() - t0
         rows_done += len(rows) * w.B * w.Hkv
-        flops_done += 4.0 * w.d * len(rows) * w.B * w.Hkv * (w.Lc + w.Lcur)
-        if spent >= budget_s or len(rows) == total_rows:
+        start += len(rows)
+        if spent >= budget_s:
             break
-        n = min(total_rows, n * 2)
+        n *= 2
     blas = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
     cores = blas or os.cpu_count()
     all_rows = total_rows * w.B * w.Hkv

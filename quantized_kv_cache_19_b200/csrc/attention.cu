@@ -19,16 +19,19 @@
 //
 // One CTA computes 128 packed query rows (the Hq/Hkv query heads of one KV head; row =
 // head_in_group * Lq + i) against every key of its (batch, KV head); tiles of N keys
-// (N = 128, or 64 with four groups). Warp roles (8 warps):
-//   warp 0     allocates tensor memory; lane 0 issues tcgen05.mma / tcgen05.commit,
-//              lane 1 issues bulk (TMA-engine) copies of packed tiles (codes and step/zero-point of
-//              N keys, K and V) into a 2-stage ring;
-//   warps 1-3  unpack K codes to bf16 integers, dequantise V to bf16 (128-byte-swizzled operand
-//              tiles, 2-slot rings) and write per-key constants (a, z, step^2); for current tiles
-//              they copy K_cur / V_cur into the operand tiles;
-//   warps 4-7  one query row per thread: Q row statistics and a bf16 copy of Q into TMEM; per tile
-//              read S from TMEM (releasing it at once), form the corrected scores, online softmax in
-//              base 2 with lazy rescaling of O, P (bf16) into TMEM; finally O / l and LSE.
+// (N = 128, or 64 with four groups). Four warpgroups, registers rebalanced with setmaxnreg:
+//   WG0      warp 0: allocates tensor memory; one thread runs a non-blocking issue loop that
+//            starts the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point of N
+//            keys, K and V) into a 4-stage ring, and every tcgen05.mma / tcgen05.commit, each as
+//            soon as its own barriers allow. Warps 1-3: K operand tiles (codes unpacked to bf16
+//            integers, 128-byte swizzle, 2-slot ring) and the per-key constants (a, z, step^2);
+//            for current tiles, a copy of K_cur.
+//   WG1/WG2  softmax, one query row per thread, WG1 on the first half of every key tile and WG2
+//            on the second: Q row statistics and a bf16 copy of Q into TMEM; per tile read S from
+//            TMEM (releasing it at once), form the corrected scores, exchange the row max through
+//            shared memory, online softmax in base 2 with lazy rescaling of O (each half rescales
+//            half of O's columns), P (bf16) into TMEM; finally O / l and LSE.
+//   WG3      V operand tiles: dequantised to bf16; for current tiles, a copy of V_cur.
 // Tensor memory (512 columns): O [0, d), Q [128, 128 + d/2), P [192, 192 + N/2),
 // S [256, 256 + groups * N) (cached tiles; current tiles use the first N columns).
 // Every mbarrier wait is bounded; on timeout the CTA records QKV_ERR_TIMEOUT in the library's
@@ -37,13 +40,15 @@
 #include "qkv_internal.h"
 #include "qkv_jensen.cuh"
 
+#include <type_traits>
+
 namespace qkv {
 namespace {
 
 constexpr int kBM = 128;                     // query rows per CTA (MMA M)
-constexpr int kThreads = 256;
-constexpr int kProducerWarps = 3;
-constexpr int kStages = 2;                   // packed-tile ring
+constexpr int kThreads = 512;                 // four warpgroups
+constexpr int kRegProducer = 96, kRegSoftmax = 160;   // 2 * 96 + 2 * 160 = 512 = 4 * 128 at launch
+constexpr int kStages = 4;                   // packed-tile ring (3 tiles of prefetch)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when the max grows by more
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColQ = 128, kColP = 192, kColS = 256;
@@ -66,12 +71,15 @@ struct Cfg {
   static constexpr int G = D / NG;                       // channels per group
   static constexpr uint32_t kTile = N * D * 2;           // bf16 operand tile
   static constexpr uint32_t kCodes = N * D * BITS / 8;   // packed codes of one tile
-  static constexpr uint32_t kKconst = N * NG * 16;       // per-key constants of one tile
+  static constexpr int NGH = (NG + 1) / 2;               // float4s of squared steps per key pair
+  // per-key constants of one tile: for each key pair q and group g, float4 (a_2q, a_2q+1, z_2q,
+  // z_2q+1); then for each pair, NGH float4 of squared steps (g even: x,y; g odd: z,w)
+  static constexpr uint32_t kKconst = (N / 2) * (NG + NGH) * 16;
   static constexpr uint32_t kDblk = N * 128;             // bytes between 64-channel blocks
 };
 
 struct Layout {
-  uint32_t kt, vt, pk, kc, bars, misc, total, stage, meta;
+  uint32_t kt, vt, pk, kc, xc, bars, misc, total, stage, meta;
 };
 
 template <int D, int BITS, int NG>
@@ -84,10 +92,17 @@ __host__ __device__ inline Layout make_layout(int meta_bytes) {
   L.vt = L.kt + 2 * C::kTile;
   L.pk = L.vt + 2 * C::kTile;
   L.kc = L.pk + kStages * L.stage;
-  L.bars = L.kc + 2 * C::kKconst;
+  L.xc = L.kc + 2 * C::kKconst;            // row-max exchange [2][2][128] and row-sum [2][128]
+  L.bars = L.xc + (4 + 2) * kBM * 4;
   L.misc = L.bars + B_COUNT * 8;
   L.total = L.misc + 16;
   return L;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -96,8 +111,7 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Non-blocking bounded spin used by the two single-lane roles that share warp 0, so that one lane
-// never parks the warp while the other has work.
+// Non-blocking bounded spin of the single issuing thread of warp 0.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -108,20 +122,6 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
-}
-__device__ __forceinline__ bool lane_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
-  if (mbar_test(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_test(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
-      *abort_flag = 1;
-      atomicCAS(status, 0, -5);
-      return false;
-    }
-  }
 }
 
 // 16 bf16x2 words (32 channels) of bf16 integers 128 + code from 32 packed codes.
@@ -168,7 +168,8 @@ __device__ __forceinline__ void dequant32(const uint8_t* codes, float step, floa
         const uint32_t s = sh >= 0 ? (w << sh) : (w >> (-sh));
         const float lo = __uint_as_float((s & (3u << 19)) | 0x3F800000u);   // 1 + c/16
         const float hi = __uint_as_float((s & (3u << 21)) | 0x3F800000u);   // 1 + c/4
-        out[h * 8 + p] = pack_bf16x2(fmaf(s16, lo, c16), fmaf(s4, hi, c4));
+        const float2 x = __ffma2_rn(make_float2(s16, s4), make_float2(lo, hi), make_float2(c16, c4));
+        out[h * 8 + p] = pack_bf16x2(x.x, x.y);
       }
     }
   } else {
@@ -184,7 +185,8 @@ __device__ __forceinline__ void dequant32(const uint8_t* codes, float step, floa
         const uint32_t s = sh >= 0 ? (w << sh) : (w >> (-sh));
         const float lo = __uint_as_float((s & (0xFu << 15)) | 0x3F800000u);  // 1 + c/256
         const float hi = __uint_as_float((s & (0xFu << 19)) | 0x3F800000u);  // 1 + c/16
-        out[h * 4 + p] = pack_bf16x2(fmaf(s256, lo, c256), fmaf(s16, hi, c16));
+        const float2 x = __ffma2_rn(make_float2(s256, s16), make_float2(lo, hi), make_float2(c256, c16));
+        out[h * 4 + p] = pack_bf16x2(x.x, x.y);
       }
     }
   }
@@ -215,21 +217,94 @@ __device__ __forceinline__ void load_meta(const uint8_t* meta, int idx, float& s
   }
 }
 
+// Copies `valid` rows (of N) of bf16 [row][D] from global memory into a [D/64][N][64] swizzled tile;
+// rows beyond `valid` become zero. NT threads, kIters (key, 32-channel block) items each.
+template <int D, int N, int kIters, int NT>
+__device__ __forceinline__ void copy_rows(const uint4* src, uint8_t* tile, int valid, int t) {
+  constexpr int kItems = N * (D / 32);
+  uint4 a[kIters][4];
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int it = t + NT * i, key = it / (D / 32), blk = it % (D / 32);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      a[i][e] = (it < kItems && key < valid) ? src[key * (D / 8) + blk * 4 + e] : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < kIters; ++i) {
+    const int it = t + NT * i, key = it / (D / 32), blk = it % (D / 32);
+    if (it >= kItems) break;
+    uint32_t v[16];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[4 * e] = a[i][e].x; v[4 * e + 1] = a[i][e].y; v[4 * e + 2] = a[i][e].z; v[4 * e + 3] = a[i][e].w;
+    }
+    store32<N>(tile, key, blk, v);
+  }
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+template <int NC>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t* r) {
+  static_assert(NC % 16 == 0, "");
+#pragma unroll
+  for (int c = 0; c < NC; c += 32) {
+    if (c + 32 <= NC) {
+      uint32_t t[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) t[k] = r[c + k];
+      tmem_st32(taddr + c, t);
+    } else {
+      tmem_st16(taddr + c, r + c);
+    }
+  }
+}
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <int D, int BITS, int NG>
 __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const AttnParams p) {
   using C = Cfg<D, BITS, NG>;
   constexpr int N = C::N;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  constexpr int NH = N / 2;                   // keys of a tile per softmax warpgroup
+  constexpr int kItems = N * (D / 32);        // (key, 32-channel block) items of one tile
+  constexpr int kItersV = kItems / 128;       // per V-producer thread (128 threads)
+  constexpr int kItersK = (kItems + 95) / 96; // per K-producer thread (96 threads)
+  static_assert(kItems % 128 == 0, "tile items must split evenly over a warpgroup");
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // 1024-byte alignment (128B-swizzle atoms) by offsetting the shared array itself, so that the
+  // compiler keeps every access in the shared address space.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const Layout L = make_layout<D, BITS, NG>(p.meta_f16 ? 2 : 4);
   const uint32_t bar0 = smem_u32(smem + L.bars);
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc + 4);
   float4* kconst = reinterpret_cast<float4*>(smem + L.kc);
+  float* xmax = reinterpret_cast<float*>(smem + L.xc);        // [tile parity][half][row]
+  float* xsum = xmax + 4 * kBM;                                // [half][row]
 
   const int warp = threadIdx.x >> 5;
+  const int wg = warp >> 2;
   const int lane = threadIdx.x & 31;
   const int m_tile = blockIdx.x;
   const int bh = blockIdx.y;
@@ -254,11 +329,11 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     *abort_flag = 0;
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_PK_EMPTY || i == B_PK_EMPTY + 1 || i == B_KH_FULL || i == B_KH_FULL + 1 ||
-          i == B_VH_FULL || i == B_VH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1)
-        cnt = kProducerWarps;
+      if (i == B_KH_FULL || i == B_KH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1) cnt = 3;
+      if (i == B_VH_FULL || i == B_VH_FULL + 1) cnt = 4;
       if (i == B_KC_EMPTY || i == B_KC_EMPTY + 1 || i == B_S_FREE || i == B_P_FULL || i == B_Q_FULL)
-        cnt = 4;                                   // softmax warps
+        cnt = 8;                                   // both softmax warpgroups
+      if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = 7;   // K and V producer warps
       mbar_init(bar(i), cnt);
     }
     mbar_init_fence();
@@ -269,37 +344,43 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (wg == 0 && warp == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
+      // -------------------------------------------- bulk-copy and MMA issue loop (one thread)
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBM, N, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t tm_q = tmem + kColQ, tm_o = tmem + kColO, tm_p = tmem + kColP;
       const uint32_t tm_s = tmem + kColS;
-      auto issue_pv = [&](int i) -> bool {
-        const int sb = i & 1, n = i >> 1;
-        if (!lane_wait(bar(B_P_FULL), i & 1, abort_flag, p.status)) return false;
-        if (!lane_wait(bar(B_VH_FULL + sb), n & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t vbase = smem_u32(smem + L.vt + sb * C::kTile);
-#pragma unroll
-        for (int kk = 0; kk < N / 16; ++kk) {
-          // V tile [d/64][N keys][64], 128B swizzle, MN-major: 16 keys per step (two 1024-byte
-          // atoms), LBO = next 64 channels, SBO = next 8 keys.
-          const uint64_t desc = smem_desc_sw128(vbase + kk * 2048u, C::kDblk, 1024u);
-          mma_ts(tm_o, tm_p + kk * 8u, desc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+      const int64_t row_codes = D * BITS / 8;
+      const int64_t row_meta = static_cast<int64_t>(NG) * 2 * (p.meta_f16 ? 2 : 4);
+      int next_load = 0, next_s = 0, next_pv = 0;
+      bool q_ready = false;
+      long long t_idle = clock64();
+      while (next_pv < T) {
+        bool progress = false;
+        // Bulk copies of the next cached tile, as far ahead as the stage ring allows.
+        if (next_load < Tc && next_load < next_s + kStages) {
+          const int s = next_load % kStages, k = next_load / kStages;
+          if (mbar_test(bar(B_PK_EMPTY + s), (k & 1) ^ 1)) {
+            const uint32_t dst = smem_u32(smem + L.pk + s * L.stage);
+            const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(next_load) * N;
+            const uint32_t fb = bar(B_PK_FULL + s);
+            mbar_arrive_expect_tx(fb, 2 * (C::kCodes + L.meta));
+            bulk_g2s(dst, p.k_codes + row0 * row_codes, C::kCodes, fb);
+            bulk_g2s(dst + C::kCodes, static_cast<const uint8_t*>(p.k_meta) + row0 * row_meta, L.meta, fb);
+            bulk_g2s(dst + C::kCodes + L.meta, p.v_codes + row0 * row_codes, C::kCodes, fb);
+            bulk_g2s(dst + 2 * C::kCodes + L.meta,
+                     static_cast<const uint8_t*>(p.v_meta) + row0 * row_meta, L.meta, fb);
+            ++next_load;
+            progress = true;
+          }
         }
-        tc_commit(bar(B_VH_EMPTY + sb));
-        tc_commit(bar(B_PV_DONE));
-        return true;
-      };
-      bool ok = T > 0 && lane_wait(bar(B_Q_FULL), 0, abort_flag, p.status);
-      if (ok) {
-        tc_fence_after();
-        for (int j = 0; j < T && ok; ++j) {
-          const int sb = j & 1, n = j >> 1;
-          if (!lane_wait(bar(B_KH_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
-          if (j > 0 && !lane_wait(bar(B_S_FREE), (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (!q_ready) q_ready = mbar_test(bar(B_Q_FULL), 0);
+        // S_j = Q K_j^T once K_j is in smem and the softmax has read S_{j-1}.
+        if (q_ready && next_s < T && mbar_test(bar(B_KH_FULL + (next_s & 1)), (next_s >> 1) & 1) &&
+            (next_s == 0 || mbar_test(bar(B_S_FREE), (next_s - 1) & 1))) {
+          const int j = next_s, sb = j & 1;
           tc_fence_after();
           const uint32_t kbase = smem_u32(smem + L.kt + sb * C::kTile);
           // K tile [d/64][N keys][64], 128B swizzle, K-major: 16 channels per step (32 bytes inside
@@ -322,81 +403,101 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           }
           tc_commit(bar(B_KH_EMPTY + sb));
           tc_commit(bar(B_S_FULL));
-          if (j >= 1) ok = issue_pv(j - 1);
+          ++next_s;
+          progress = true;
         }
-        if (ok) issue_pv(T - 1);
+        // O += P_i V_i once the softmax wrote P_i and V_i is in smem.
+        if (next_pv < next_s && mbar_test(bar(B_P_FULL), next_pv & 1) &&
+            mbar_test(bar(B_VH_FULL + (next_pv & 1)), (next_pv >> 1) & 1)) {
+          const int i = next_pv, sb = i & 1;
+          tc_fence_after();
+          const uint32_t vbase = smem_u32(smem + L.vt + sb * C::kTile);
+#pragma unroll
+          for (int kk = 0; kk < N / 16; ++kk) {
+            // V tile [d/64][N keys][64], 128B swizzle, MN-major: 16 keys per step (two 1024-byte
+            // atoms), LBO = next 64 channels, SBO = next 8 keys.
+            const uint64_t desc = smem_desc_sw128(vbase + kk * 2048u, C::kDblk, 1024u);
+            mma_ts(tm_o, tm_p + kk * 8u, desc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar(B_VH_EMPTY + sb));
+          tc_commit(bar(B_PV_DONE));
+          ++next_pv;
+          progress = true;
+        }
+        if (progress) {
+          t_idle = clock64();
+        } else {
+          __nanosleep(32);   // leave the issue slots of this sub-partition to the other warps
+          if (*abort_flag) break;
+          if (clock64() - t_idle > kWaitLimitCycles) {
+            *abort_flag = 1;
+            atomicCAS(p.status, 0, -5);
+            break;
+          }
+        }
       }
-      // Never free tensor memory under a running MMA.
+      // Never free tensor memory under a running MMA, never leave with copies in flight.
       tc_commit(bar(B_DRAIN));
       mbar_wait_drain(bar(B_DRAIN), 0);
-    } else if (lane == 1) {
-      // ---------------------------------------------------------------- bulk-copy producer
-      const int64_t row_codes = D * BITS / 8;
-      const int64_t row_meta = static_cast<int64_t>(NG) * 2 * (p.meta_f16 ? 2 : 4);
-      int issued = 0;
-      for (int jc = 0; jc < Tc; ++jc) {
-        const int s = jc % kStages, k = jc / kStages;
-        if (!lane_wait(bar(B_PK_EMPTY + s), (k & 1) ^ 1, abort_flag, p.status)) break;
-        const uint32_t dst = smem_u32(smem + L.pk + s * L.stage);
-        const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(jc) * N;
-        const uint32_t fb = bar(B_PK_FULL + s);
-        mbar_arrive_expect_tx(fb, 2 * (C::kCodes + L.meta));
-        bulk_g2s(dst, p.k_codes + row0 * row_codes, C::kCodes, fb);
-        bulk_g2s(dst + C::kCodes, static_cast<const uint8_t*>(p.k_meta) + row0 * row_meta, L.meta, fb);
-        bulk_g2s(dst + C::kCodes + L.meta, p.v_codes + row0 * row_codes, C::kCodes, fb);
-        bulk_g2s(dst + 2 * C::kCodes + L.meta, static_cast<const uint8_t*>(p.v_meta) + row0 * row_meta,
-                 L.meta, fb);
-        ++issued;
-      }
-      // Never leave the CTA with copies in flight: wait for the last use of every stage.
-      for (int s = 0; s < kStages && s < issued; ++s) {
-        const int last = ((issued - 1 - s) / kStages) * kStages + s;
+      for (int s = 0; s < kStages && s < next_load; ++s) {
+        const int last = ((next_load - 1 - s) / kStages) * kStages + s;
         mbar_wait_drain(bar(B_PK_FULL + s), (last / kStages) & 1);
       }
     }
     __syncwarp();
-  } else if (warp <= kProducerWarps) {
-    // ---------------------------------------------------------------- operand producers
+  } else if (wg == 0) {
+    // ---------------------------------------------------------------- K operand tiles (warps 1-3)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = threadIdx.x - 32;
-    constexpr int kItems = N * (D / 32);     // (key, 32-channel block) items per tile
-    constexpr int kNT = kProducerWarps * 32;
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* kt = smem + L.kt + sb * C::kTile;
-      uint8_t* vt = smem + L.vt + sb * C::kTile;
+      if (!warp_wait(bar(B_KH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
       if (j < Tc) {
         const int s = j % kStages, k = j / kStages;
         const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
         const int valid = static_cast<int>(rem < N ? rem : N);
-        const uint8_t* st = smem + L.pk + s * L.stage;
-        const uint8_t* kcodes = st;
-        const uint8_t* kmeta = st + C::kCodes;
-        const uint8_t* vcodes = st + C::kCodes + L.meta;
-        const uint8_t* vmeta = st + 2 * C::kCodes + L.meta;
+        const uint8_t* kcodes = smem + L.pk + s * L.stage;
+        const uint8_t* kmeta = kcodes + C::kCodes;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
-        if (!warp_wait(bar(B_KH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
         if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
-        float4* kc = kconst + sb * (N * NG);
-        for (int it = t; it < kItems; it += kNT) {
-          const int key = it / (D / 32), blk = it % (D / 32);
-          const int g = (blk * 32) / C::G;
+        float4* kc = kconst + sb * (C::kKconst / 16);
+        using CodeVec = typename std::conditional<BITS == 2, uint2, uint4>::type;
+        CodeVec cv[kItersK];
+#pragma unroll
+        for (int i = 0; i < kItersK; ++i) {
+          const int it = t + 96 * i, key = it / (D / 32), blk = it % (D / 32);
+          if (it < kItems)
+            cv[i] = *reinterpret_cast<const CodeVec*>(kcodes + key * (D * BITS / 8) + blk * (4 * BITS));
+        }
+#pragma unroll
+        for (int i = 0; i < kItersK; ++i) {
+          const int it = t + 96 * i, key = it / (D / 32), blk = it % (D / 32);
+          if (it >= kItems) break;
           uint32_t v[16];
           if (key < valid) {
-            unpack_codes32<BITS>(kcodes + key * (D * BITS / 8) + blk * (4 * BITS), v);
+            unpack_codes32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), v);
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
           store32<N>(kt, key, blk, v);
           if ((blk * 32) % C::G == 0) {
-            float4 c = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int g = (blk * 32) / C::G;
+            float a = 0.f, z = 0.f, d2 = 0.f;
             if (key < valid) {
               float step, zp;
               if (p.meta_f16) load_meta<true>(kmeta, key * NG + g, step, zp);
               else load_meta<false>(kmeta, key * NG + g, step, zp);
-              c = make_float4(step * p.scale_log2, (zp - 128.f * step) * p.scale_log2, step * step, 0.f);
+              a = step * p.scale_log2;
+              z = (zp - 128.f * step) * p.scale_log2;
+              d2 = step * step;
             }
-            kc[key * NG + g] = c;
+            float* az = reinterpret_cast<float*>(kc + (key >> 1) * NG + g);
+            az[key & 1] = a;
+            az[2 + (key & 1)] = z;
+            float* dd = reinterpret_cast<float*>(kc + (N / 2) * NG + (key >> 1) * C::NGH + (g >> 1));
+            dd[(g & 1) * 2 + (key & 1)] = d2;
           }
         }
         fence_async_smem();
@@ -404,17 +505,50 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         if (lane == 0) {
           mbar_arrive(bar(B_KH_FULL + sb));
           mbar_arrive(bar(B_KC_FULL + sb));
+          mbar_arrive(bar(B_PK_EMPTY + s));
         }
-        if (!warp_wait(bar(B_VH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
-        for (int it = t; it < kItems; it += kNT) {
-          const int key = it / (D / 32), blk = it % (D / 32);
+      } else {
+        const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
+        const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
+        const uint4* src = reinterpret_cast<const uint4*>(p.K_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
+        copy_rows<D, N, kItersK, 96>(src, kt, valid, t);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_KH_FULL + sb));
+      }
+    }
+  } else if (wg == 3) {
+    // ---------------------------------------------------------------- V operand tiles
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
+    const int t = threadIdx.x - 384;
+    for (int j = 0; j < T; ++j) {
+      const int sb = j & 1, n = j >> 1;
+      uint8_t* vt = smem + L.vt + sb * C::kTile;
+      if (!warp_wait(bar(B_VH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+      if (j < Tc) {
+        const int s = j % kStages, k = j / kStages;
+        const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
+        const int valid = static_cast<int>(rem < N ? rem : N);
+        const uint8_t* vcodes = smem + L.pk + s * L.stage + C::kCodes + L.meta;
+        const uint8_t* vmeta = vcodes + C::kCodes;
+        if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
+        using CodeVec = typename std::conditional<BITS == 2, uint2, uint4>::type;
+        CodeVec cv[kItersV];
+        float st[kItersV], zp[kItersV];
+#pragma unroll
+        for (int i = 0; i < kItersV; ++i) {
+          const int it = t + 128 * i, key = it / (D / 32), blk = it % (D / 32);
           const int g = (blk * 32) / C::G;
+          cv[i] = *reinterpret_cast<const CodeVec*>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS));
+          if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, st[i], zp[i]);
+          else load_meta<false>(vmeta, key * NG + g, st[i], zp[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < kItersV; ++i) {
+          const int it = t + 128 * i, key = it / (D / 32), blk = it % (D / 32);
           uint32_t v[16];
           if (key < valid) {
-            float step, zp;
-            if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, step, zp);
-            else load_meta<false>(vmeta, key * NG + g, step, zp);
-            dequant32<BITS>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS), step, zp, v);
+            dequant32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), st[i], zp[i], v);
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0u;
@@ -430,41 +564,17 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
-        const int64_t row0 = static_cast<int64_t>(bh) * p.Lcur + t0;
-        const uint4* ksrc = reinterpret_cast<const uint4*>(p.K_cur) + row0 * (D / 8);
-        const uint4* vsrc = reinterpret_cast<const uint4*>(p.V_cur) + row0 * (D / 8);
-        bool ok = true;
-        for (int pass = 0; pass < 2 && ok; ++pass) {
-          if (!warp_wait(bar((pass ? B_VH_EMPTY : B_KH_EMPTY) + sb), (n & 1) ^ 1, abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          const uint4* src = pass ? vsrc : ksrc;
-          uint8_t* dst = pass ? vt : kt;
-          for (int it = t; it < kItems; it += kNT) {
-            const int key = it / (D / 32), blk = it % (D / 32);
-            uint32_t v[16];
-            if (key < valid) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const uint4 a = src[key * (D / 8) + blk * 4 + i];
-                v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = 0u;
-            }
-            store32<N>(dst, key, blk, v);
-          }
-          fence_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar((pass ? B_VH_FULL : B_KH_FULL) + sb));
-        }
-        if (!ok) break;
+        const uint4* src = reinterpret_cast<const uint4*>(p.V_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
+        copy_rows<D, N, kItersV, 128>(src, vt, valid, t);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_VH_FULL + sb));
       }
     }
   } else {
-    // ---------------------------------------------------------------- softmax / epilogue
+    // ---------------------------------------------------------------- softmax / epilogue (WG1, WG2)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegSoftmax));
+    const int half = wg - 1;                   // which half of every key tile
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -473,19 +583,19 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     const int64_t hq = static_cast<int64_t>(h) * p.r + (valid_row ? R / p.Lq : 0);
     const int64_t qi = valid_row ? R % p.Lq : 0;
     const int64_t out_row = (static_cast<int64_t>(b) * p.Hq + hq) * p.Lq + qi;
+    const int kbase_h = half * NH;             // first key of this warpgroup's half of a tile
 
-    // Q row: group sums of q (what the codes multiply), correction weights, bf16 copy into TMEM.
+    // Q row: group sums of q (what the codes multiply), correction weights; this half's columns of
+    // the bf16 copy of Q go into TMEM.
     float w[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
     float qs[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
     {
       const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * 2;
-      uint32_t qp[D / 2];
+      uint32_t qp[D / 4];
       if (valid_row) {
         query_group_weights<D>(qrow, false, C::G, p.wcoef_log2, w);
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
-          const uint4 u = reinterpret_cast<const uint4*>(qrow)[c8];
-          qp[4 * c8] = u.x; qp[4 * c8 + 1] = u.y; qp[4 * c8 + 2] = u.z; qp[4 * c8 + 3] = u.w;
           float x[8];
           load_q8(qrow, false, c8, x);
           float acc = 0.f;
@@ -495,17 +605,16 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           for (int g = 0; g < NG; ++g)
             if (g == (c8 * 8) / C::G) qs[g] += acc;
         }
+#pragma unroll
+        for (int c8 = 0; c8 < D / 16; ++c8) {
+          const uint4 u = reinterpret_cast<const uint4*>(qrow)[half * (D / 16) + c8];
+          qp[4 * c8] = u.x; qp[4 * c8 + 1] = u.y; qp[4 * c8 + 2] = u.z; qp[4 * c8 + 3] = u.w;
+        }
       } else {
 #pragma unroll
-        for (int k = 0; k < D / 2; ++k) qp[k] = 0u;
+        for (int k = 0; k < D / 4; ++k) qp[k] = 0u;
       }
-#pragma unroll
-      for (int c = 0; c < D / 2; c += 32) {
-        uint32_t chunk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) chunk[k] = qp[c + k];
-        tmem_st32(tmem + lane_off + kColQ + c, chunk);
-      }
+      tmem_st<D / 4>(tmem + lane_off + kColQ + half * (D / 4), qp);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -516,42 +625,54 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       for (int g = 0; g < kMaxGroups; ++g) w[g] = 0.f;
     }
 
-    float m_run = -INFINITY;   // max used for the exponentials so far (log2 units)
-    float l_run = 0.f;
+    float m_run = -INFINITY;   // max used for the exponentials so far (log2 units), same in both halves
+    float l_run = 0.f;         // this half's part of the softmax denominator
+    float2 qs2[NG], nw2[NG];   // broadcast pairs of the row's group sums and -correction weights
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      qs2[g] = make_float2(qs[g], qs[g]);
+      nw2[g] = make_float2(-w[g], -w[g]);
+    }
+    const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int j = 0; j < T && ok; ++j) {
       const int sb = j & 1, n = j >> 1;
       const bool cached = j < Tc;
       if (!warp_wait(bar(B_S_FULL), j & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tm_s = tmem + lane_off + kColS;
-      float s[N];
+      const uint32_t tm_s = tmem + lane_off + kColS + kbase_h;
+      float2 s2[NH / 2];         // scores of this half's key pairs (log2 units)
+      int valid;                 // keys of the whole tile that count for this row
       if (cached) {
         const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
-        const int valid = static_cast<int>(rem < N ? rem : N);
+        valid = static_cast<int>(rem < N ? rem : N);
         if (!warp_wait(bar(B_KC_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
-        const float4* kc = kconst + sb * (N * NG);
+        const float4* az = kconst + sb * (C::kKconst / 16);
+        const float4* dd = az + (N / 2) * NG;
 #pragma unroll
-        for (int c = 0; c < N; c += 32) {
+        for (int c = 0; c < NH; c += 16) {
+          uint32_t r[NG][16];
 #pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            uint32_t r[32];
-            tmem_ld32(tm_s + g * N + c, r);
-            tmem_wait_ld();
+          for (int g = 0; g < NG; ++g) tmem_ld16(tm_s + g * N + c, r[g]);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-              const float4 cst = kc[(c + k) * NG + g];
-              const float part = fmaf(cst.x, __uint_as_float(r[k]), cst.y * qs[g]);
-              s[c + k] = g == 0 ? part : s[c + k] + part;
+          for (int q = 0; q < 8; ++q) {
+            const int pq = (kbase_h + c) / 2 + q;
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int gh = 0; gh < C::NGH; ++gh) {
+              const float4 d = dd[pq * C::NGH + gh];
+              acc = __ffma2_rn(make_float2(d.x, d.y), nw2[2 * gh], acc);
+              if (2 * gh + 1 < NG) acc = __ffma2_rn(make_float2(d.z, d.w), nw2[2 * gh + 1], acc);
             }
-          }
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            float d2[kMaxGroups];
-#pragma unroll
-            for (int g = 0; g < kMaxGroups; ++g) d2[g] = g < NG ? kc[(c + k) * NG + g].z : 0.f;
-            const float t = s[c + k] - jensen_term(w, d2, NG);
-            s[c + k] = (c + k) < valid ? t : -INFINITY;
+            for (int g = 0; g < NG; ++g) {
+              const float4 a = az[pq * NG + g];
+              acc = __ffma2_rn(make_float2(a.z, a.w), qs2[g], acc);
+              acc = __ffma2_rn(make_float2(a.x, a.y),
+                               make_float2(__uint_as_float(r[g][2 * q]), __uint_as_float(r[g][2 * q + 1])), acc);
+            }
+            s2[c / 2 + q] = acc;
           }
         }
         tc_fence_before();
@@ -567,23 +688,40 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           const int64_t c = qi + (p.Lcur - p.Lq) - t0 + 1;  // keys this row may see
           lim = c < lim ? c : lim;
         }
-        const int valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
+        valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
 #pragma unroll
-        for (int c = 0; c < N; c += 32) {
+        for (int c = 0; c < NH; c += 32) {
           uint32_t r[32];
           tmem_ld32(tm_s + c, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            s[c + k] = (c + k) < valid ? __uint_as_float(r[k]) * p.scale_log2 : -INFINITY;
+          for (int q = 0; q < 16; ++q)
+            s2[c / 2 + q] = __fmul2_rn(make_float2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), scale2);
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_S_FREE));
       }
-      float m_tile = -INFINITY;
+      if (valid < kbase_h + NH) {
 #pragma unroll
-      for (int k = 0; k < N; ++k) m_tile = fmaxf(m_tile, s[k]);
+        for (int q = 0; q < NH / 2; ++q) {
+          if (kbase_h + 2 * q >= valid) s2[q].x = -INFINITY;
+          if (kbase_h + 2 * q + 1 >= valid) s2[q].y = -INFINITY;
+        }
+      }
+      // Row max of this half (four chains of 3-input maxima), then of the tile via shared memory.
+      float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < NH / 2; q += 4) {
+        m0 = fmax3(m0, s2[q].x, s2[q].y);
+        m1 = fmax3(m1, s2[q + 1].x, s2[q + 1].y);
+        m2 = fmax3(m2, s2[q + 2].x, s2[q + 2].y);
+        m3 = fmax3(m3, s2[q + 3].x, s2[q + 3].y);
+      }
+      const float m_half = fmax3(fmaxf(m0, m1), m2, m3);
+      xmax[((j & 1) * 2 + half) * kBM + row] = m_half;
+      named_sync(1, 256);
+      const float m_tile = fmaxf(m_half, xmax[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
       // Lazy rescaling: keep the old max unless the new one exceeds it by the threshold.
       const bool need = (m_tile > m_run + kRescaleThreshold) ||
                         (m_run == -INFINITY && m_tile > -INFINITY);
@@ -594,59 +732,62 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         m_run = m_tile;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      uint32_t pk[N / 2];
-      float psum = 0.f;
-#pragma unroll
-      for (int k = 0; k < N / 2; ++k) {
-        const float p0 = ex2(s[2 * k] - m_use);
-        const float p1 = ex2(s[2 * k + 1] - m_use);
-        psum += p0 + p1;
-        pk[k] = pack_bf16x2(p0, p1);
-      }
-      l_run += psum;
       if (j > 0) {
         // P and O must not be touched while the previous P.V is in flight.
         if (!warp_wait(bar(B_PV_DONE), (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
-          const uint32_t tm_o = tmem + lane_off + kColO;
+          const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
+          const float2 f2 = make_float2(factor, factor);
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
+          for (int c = 0; c < D / 2; c += 32) {
             uint32_t r[32];
             tmem_ld32(tm_o + c, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * factor);
+            for (int k = 0; k < 32; k += 2) {
+              const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), f2);
+              r[k] = __float_as_uint(o2.x);
+              r[k + 1] = __float_as_uint(o2.y);
+            }
             tmem_st32(tm_o + c, r);
           }
         }
       }
+      const float2 mneg = make_float2(-m_use, -m_use);
+      float2 psum = make_float2(0.f, 0.f);
+      uint32_t pk[NH / 2];
 #pragma unroll
-      for (int c = 0; c < N / 2; c += 32) {
-        uint32_t chunk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) chunk[k] = pk[c + k];
-        tmem_st32(tmem + lane_off + kColP + c, chunk);
+      for (int k = 0; k < NH / 2; ++k) {
+        const float2 e = __fadd2_rn(s2[k], mneg);
+        const float2 pp = make_float2(ex2(e.x), ex2(e.y));
+        psum = __fadd2_rn(psum, pp);
+        pk[k] = pack_bf16x2(pp.x, pp.y);
       }
+      tmem_st<NH / 2>(tmem + lane_off + kColP + kbase_h / 2, pk);
+      l_run += psum.x + psum.y;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_P_FULL));
     }
 
-    // Epilogue: O / l and LSE.
+    // Epilogue: combine the two halves' denominators, O / l (each half writes half the columns), LSE.
     bool have_o = false;
     if (ok && T > 0) {
       have_o = warp_wait(bar(B_PV_DONE), (T - 1) & 1, abort_flag, p.status);
       tc_fence_after();
     }
-    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-    uint8_t* orow = static_cast<uint8_t*>(p.O) + out_row * D * 2;
+    xsum[half * kBM + row] = l_run;
+    named_sync(1, 256);
+    const float l_tot = l_run + xsum[(half ^ 1) * kBM + row];
+    const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+    uint8_t* orow = static_cast<uint8_t*>(p.O) + out_row * D * 2 + half * D;
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
+    for (int c = 0; c < D / 2; c += 32) {
       uint32_t r[32];
       if (have_o) {
-        tmem_ld32(tmem + lane_off + kColO + c, r);
+        tmem_ld32(tmem + lane_off + kColO + half * (D / 2) + c, r);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -665,9 +806,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         }
       }
     }
-    if (valid_row) {
+    if (valid_row && half == 0) {
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      p.LSE[out_row] = l_run > 0.f ? (m_use + __log2f(l_run)) * 0.69314718055994530942f : -INFINITY;
+      p.LSE[out_row] = l_tot > 0.f ? (m_use + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
     }
   }
 
