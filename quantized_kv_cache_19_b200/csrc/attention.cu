@@ -9,21 +9,23 @@
 //
 // Cached-key scores are computed from the integer codes, not from bf16-rounded keys: with
 // x_hat = zp_g + step_g * code per group g,
-//     q . x_hat_j = sum_g step_jg * (q_g . code_jg) + zp_jg * sum(q_g).
-// The tensor core computes P'_g = q_g . (128 + code_jg) exactly (small integers are exact in bf16,
-// fp32 accumulate) into one TMEM accumulator per group; the softmax warps then form, in fp32,
-//     t_ij = sum_g [a_jg P'_ijg + z_jg qs_ig] - b_ij      (log2 units)
-// with a = step * scale * log2 e, z = (zp - 128 step) * scale * log2 e, qs_ig = sum_{c in g} q_ic.
-// Rounding keys to bf16 instead would move the log-sum-exp by up to ~3e-2 on keys with outlier
-// channels. Values are dequantised to bf16 (x_hat in fp32, then rounded) for the P.V product.
+//     t_ij = sum_g a_jg * [ q_ig . code_jg + qs_ig * rho_jg - w_ig * sigma_jg ]    (log2 units)
+// where a = step' * scale * log2 e (step' = step, or 1 for a constant group), rho = zp / step',
+// sigma = step / (scale * log2 e), qs_ig = sum_{c in g} q_ic and w_ig = (scale^2 / 24) log2 e
+// sum_{c in g} q_ic^2 (so that a * w * sigma is the Jensen term b). The bracket is one tensor-core
+// accumulator per group: the codes are exact small integers in bf16 (fp32 accumulate), and the
+// two rank-1 terms ride on one extra 16-channel k-step per group whose operands are the row and
+// key values split into bf16 parts (hi+lo for rho, hi+mid+lo for the correction), which keeps
+// them to ~1e-5 of the zero-point term and ~1e-7 of b. The softmax then needs one FMA per group
+// per score. Rounding keys to bf16 instead would move the log-sum-exp by up to ~3e-2 on keys with
+// outlier channels. Values are dequantised to bf16 (x_hat in fp32, then rounded) for P.V.
 //
 // One CTA computes 128 packed query rows (the Hq/Hkv query heads of one KV head; row =
 // head_in_group * Lq + i) against every key of its (batch, KV head); tiles of N keys
-// (N = 128, or 64 with four groups). Four warpgroups, registers rebalanced with setmaxnreg:
-//   WG0      warp 0: allocates tensor memory; one thread runs a non-blocking issue loop that
-//            starts the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point of N
-//            keys, K and V) into a 4-stage ring, and every tcgen05.mma / tcgen05.commit, each as
-//            soon as its own barriers allow. Warps 1-3: K operand tiles (codes unpacked to bf16
+// (N = 64, or 32 with four groups). Four warpgroups, registers rebalanced with setmaxnreg:
+//   WG0      warp 0: allocates tensor memory; one thread issues, in order, S_j = Q K_j^T and then
+//            P_{j-1} V_{j-1} with precomputed descriptors (an MMA issue blocks while the tensor
+//            pipe is busy, so one lean ordered stream keeps it fed). Warps 1-3: K operand tiles (codes unpacked to bf16
 //            integers, 128-byte swizzle, 2-slot ring) and the per-key constants (a, z, step^2);
 //            for current tiles, a copy of K_cur.
 //   WG1/WG2  softmax, one query row per thread, WG1 on the first half of every key tile and WG2
@@ -31,9 +33,14 @@
 //            TMEM (releasing it at once), form the corrected scores, exchange the row max through
 //            shared memory, online softmax in base 2 with lazy rescaling of O (each half rescales
 //            half of O's columns), P (bf16) into TMEM; finally O / l and LSE.
-//   WG3      V operand tiles: dequantised to bf16; for current tiles, a copy of V_cur.
-// Tensor memory (512 columns): O [0, d), Q [128, 128 + d/2), P [192, 192 + N/2),
-// S [256, 256 + groups * N) (cached tiles; current tiles use the first N columns).
+//   WG3      V operand tiles: dequantised to bf16; for current tiles, a copy of V_cur. One lane
+//            also issues the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point of
+//            N keys, K and V) into a 3-4 stage ring, as soon as K and V are done with a stage.
+// Tensor memory (512 columns): O [0, d), Q [128, 128 + d/2), P two buffers of N/2 at 192 and 224,
+// S two buffers of groups * N at 256 and 384 (current tiles use the first N columns of a buffer).
+// With both S and P double-buffered, the softmax of tile j+1 proceeds while P_j.V_j runs; it waits
+// for the previous P.V only to rescale O (rare: lazy rescaling) and for P.V two tiles back before
+// reusing a P buffer.
 // Every mbarrier wait is bounded; on timeout the CTA records QKV_ERR_TIMEOUT in the library's
 // device status word, drains its copies and MMAs, frees tensor memory and returns.
 #include "qkv_common.cuh"
@@ -48,38 +55,46 @@ namespace {
 constexpr int kBM = 128;                     // query rows per CTA (MMA M)
 constexpr int kThreads = 512;                 // four warpgroups
 constexpr int kRegProducer = 96, kRegSoftmax = 160;   // 2 * 96 + 2 * 160 = 512 = 4 * 128 at launch
-constexpr int kStages = 4;                   // packed-tile ring (3 tiles of prefetch)
+constexpr int kStagesMax = 4;                // packed-tile ring (INT2: 4 stages, INT4: 3)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when the max grows by more
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColQ = 128, kColP = 192, kColS = 256;
+constexpr uint32_t kColO = 0, kColQ = 128, kColP = 192, kColS = 256;   // P: 2 x 32, S: 2 x 128
 constexpr uint32_t kCodeMagic = 0x43004300u;  // bf16 pair (128 + c_lo, 128 + c_hi)
 
 enum {
-  B_PK_FULL = 0, B_PK_EMPTY = B_PK_FULL + kStages,
-  B_KH_FULL = B_PK_EMPTY + kStages, B_KH_EMPTY = B_KH_FULL + 2,
+  B_PK_FULL = 0, B_PK_EMPTY = B_PK_FULL + kStagesMax,
+  B_KH_FULL = B_PK_EMPTY + kStagesMax, B_KH_EMPTY = B_KH_FULL + 2,
   B_VH_FULL = B_KH_EMPTY + 2, B_VH_EMPTY = B_VH_FULL + 2,
   B_KC_FULL = B_VH_EMPTY + 2, B_KC_EMPTY = B_KC_FULL + 2,
-  B_S_FULL = B_KC_EMPTY + 2, B_S_FREE = B_S_FULL + 1,
-  B_P_FULL = B_S_FREE + 1, B_PV_DONE = B_P_FULL + 1,
-  B_Q_FULL = B_PV_DONE + 1, B_DRAIN = B_Q_FULL + 1,
+  B_S_FULL = B_KC_EMPTY + 2, B_S_FREE = B_S_FULL + 2,
+  B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
+  B_Q_FULL = B_PV_DONE + 2, B_DRAIN = B_Q_FULL + 1,
   B_COUNT = B_DRAIN + 1
 };
 
 template <int D, int BITS, int NG>
 struct Cfg {
-  static constexpr int N = NG == 4 ? 64 : 128;          // keys per tile
+  static constexpr int N = NG == 4 ? 32 : 64;           // keys per tile (S and P double-buffered)
+  static constexpr int kSCols = (NG == 1 ? 2 : NG) * N;  // TMEM columns of one S buffer (= 128)
   static constexpr int G = D / NG;                       // channels per group
   static constexpr uint32_t kTile = N * D * 2;           // bf16 operand tile
   static constexpr uint32_t kCodes = N * D * BITS / 8;   // packed codes of one tile
-  static constexpr int NGH = (NG + 1) / 2;               // float4s of squared steps per key pair
-  // per-key constants of one tile: for each key pair q and group g, float4 (a_2q, a_2q+1, z_2q,
-  // z_2q+1); then for each pair, NGH float4 of squared steps (g even: x,y; g odd: z,w)
-  static constexpr uint32_t kKconst = (N / 2) * (NG + NGH) * 16;
+  // Score accumulators per tile: one per group, and at least two, so that consecutive MMAs of a
+  // tile go to independent accumulators (a chain into one accumulator at N = 64 runs at a third of
+  // the tensor rate). A one-group cache splits its channels over two accumulators of equal scale.
+  static constexpr int NA = NG == 1 ? 2 : NG;
+  static constexpr int GA = D / NA;                      // channels per accumulator
+  static constexpr int NAH = (NA + 1) / 2;               // float4s of scales per key pair
+  // per-key scales a of one tile: for each key pair, NAH float4 (acc even: x,y; acc odd: z,w)
+  static constexpr uint32_t kKconst = (N / 2) * NAH * 16;
+  static constexpr uint32_t kAx = NG * kBM * 32;         // row extras, [g][128 rows][16] bf16
+  static constexpr uint32_t kBx = NG * N * 32;           // key extras of one tile, [g][N][16] bf16
+  static constexpr int kStages = BITS == 2 ? 4 : 3;
   static constexpr uint32_t kDblk = N * 128;             // bytes between 64-channel blocks
 };
 
 struct Layout {
-  uint32_t kt, vt, pk, kc, xc, bars, misc, total, stage, meta;
+  uint32_t kt, vt, pk, kc, ax, bx, xc, bars, misc, total, stage, meta;
 };
 
 template <int D, int BITS, int NG>
@@ -91,8 +106,10 @@ __host__ __device__ inline Layout make_layout(int meta_bytes) {
   L.kt = 0;
   L.vt = L.kt + 2 * C::kTile;
   L.pk = L.vt + 2 * C::kTile;
-  L.kc = L.pk + kStages * L.stage;
-  L.xc = L.kc + 2 * C::kKconst;            // row-max exchange [2][2][128] and row-sum [2][128]
+  L.kc = L.pk + C::kStages * L.stage;
+  L.ax = (L.kc + 2 * C::kKconst + 127) & ~127u;
+  L.bx = L.ax + C::kAx;
+  L.xc = L.bx + 2 * C::kBx;                // row-max exchange [2][2][128] and row-sum [2][128]
   L.bars = L.xc + (4 + 2) * kBM * 4;
   L.misc = L.bars + B_COUNT * 8;
   L.total = L.misc + 16;
@@ -111,7 +128,16 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Non-blocking bounded spin of the single issuing thread of warp 0.
+// Parks the thread in hardware until the phase completes or about `ns` nanoseconds pass.
+__device__ __forceinline__ void mbar_park(uint32_t bar, uint32_t parity, uint32_t ns) {
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P1, [%0], %1, %2;\n\t}" ::"r"(bar),
+      "r"(parity), "r"(ns)
+      : "memory");
+}
+
+// Non-blocking test used by the single issuing thread of warp 0.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -124,7 +150,30 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// 16 bf16x2 words (32 channels) of bf16 integers 128 + code from 32 packed codes.
+// 16 bf16x2 words (32 channels) of the codes as exact bf16 integers: (128 + code) built in the
+// mantissa, then 128 subtracted (exact).
+__device__ __forceinline__ uint32_t bf16x2_sub128(uint32_t v) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&v);
+  x = __hsub2(x, __floats2bfloat162_rn(128.f, 128.f));
+  return *reinterpret_cast<uint32_t*>(&x);
+}
+
+// Splits x into bf16 parts: x ~ hi + mid + lo.
+__device__ __forceinline__ void split3(float x, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(hi);
+  mid = __float2bfloat16_rn(r1);
+  lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+}
+
+// 16 bf16 channels of one row of an extras tile in the no-swizzle K-major core-matrix layout
+// [row / 8][2 halves][row % 8][8].
+__device__ __forceinline__ void store_extras(uint8_t* tile, int row, const __nv_bfloat16 (&v)[16]) {
+  uint8_t* base = tile + (row >> 3) * 256 + (row & 7) * 16;
+  *reinterpret_cast<uint4*>(base) = *reinterpret_cast<const uint4*>(&v[0]);
+  *reinterpret_cast<uint4*>(base + 128) = *reinterpret_cast<const uint4*>(&v[8]);
+}
+
 template <int BITS>
 __device__ __forceinline__ void unpack_codes32(const uint8_t* codes, uint32_t (&out)[16]) {
   if constexpr (BITS == 2) {
@@ -135,7 +184,7 @@ __device__ __forceinline__ void unpack_codes32(const uint8_t* codes, uint32_t (&
       const uint32_t half = (h & 1) ? (word >> 16) : (word & 0xFFFFu);
       const uint32_t v = half | (half << 14);   // code 2p at bit 4p, code 2p+1 at bit 16+4p
 #pragma unroll
-      for (int p = 0; p < 4; ++p) out[h * 4 + p] = ((v >> (4 * p)) & 0x00030003u) | kCodeMagic;
+      for (int p = 0; p < 4; ++p) out[h * 4 + p] = bf16x2_sub128(((v >> (4 * p)) & 0x00030003u) | kCodeMagic);
     }
   } else {
     const uint4 w4 = *reinterpret_cast<const uint4*>(codes);
@@ -145,7 +194,7 @@ __device__ __forceinline__ void unpack_codes32(const uint8_t* codes, uint32_t (&
       const uint32_t half = (h & 1) ? (word >> 16) : (word & 0xFFFFu);
       const uint32_t v = half | (half << 12);   // code 2p at bit 8p, code 2p+1 at bit 16+8p
 #pragma unroll
-      for (int p = 0; p < 2; ++p) out[h * 2 + p] = ((v >> (8 * p)) & 0x000F000Fu) | kCodeMagic;
+      for (int p = 0; p < 2; ++p) out[h * 2 + p] = bf16x2_sub128(((v >> (8 * p)) & 0x000F000Fu) | kCodeMagic);
     }
   }
 }
@@ -262,18 +311,53 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld16p(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+// NC consecutive columns (a multiple of 8) of this thread's TMEM lane, from / into a register array.
 template <int NC>
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t* r) {
-  static_assert(NC % 16 == 0, "");
+  static_assert(NC % 8 == 0, "");
 #pragma unroll
-  for (int c = 0; c < NC; c += 32) {
+  for (int c = 0; c < NC;) {
     if (c + 32 <= NC) {
       uint32_t t[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) t[k] = r[c + k];
       tmem_st32(taddr + c, t);
-    } else {
+      c += 32;
+    } else if (c + 16 <= NC) {
       tmem_st16(taddr + c, r + c);
+      c += 16;
+    } else {
+      tmem_st8(taddr + c, r + c);
+      c += 8;
+    }
+  }
+}
+template <int NC>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t* r) {
+  static_assert(NC % 16 == 0, "");
+#pragma unroll
+  for (int c = 0; c < NC;) {
+    if (c + 32 <= NC) {
+      tmem_ld32p(taddr + c, r + c);
+      c += 32;
+    } else {
+      tmem_ld16p(taddr + c, r + c);
+      c += 16;
     }
   }
 }
@@ -285,6 +369,7 @@ template <int D, int BITS, int NG>
 __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const AttnParams p) {
   using C = Cfg<D, BITS, NG>;
   constexpr int N = C::N;
+  constexpr int kStages = C::kStages;
   constexpr int NH = N / 2;                   // keys of a tile per softmax warpgroup
   constexpr int kItems = N * (D / 32);        // (key, 32-channel block) items of one tile
   constexpr int kItersV = kItems / 128;       // per V-producer thread (128 threads)
@@ -300,6 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc + 4);
   float4* kconst = reinterpret_cast<float4*>(smem + L.kc);
+  uint8_t* ax = smem + L.ax;                                   // row extras (written by the softmax)
+  uint8_t* bx = smem + L.bx;                                   // key extras ring (K producers)
   float* xmax = reinterpret_cast<float*>(smem + L.xc);        // [tile parity][half][row]
   float* xsum = xmax + 4 * kBM;                                // [half][row]
 
@@ -331,7 +418,8 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       uint32_t cnt = 1;
       if (i == B_KH_FULL || i == B_KH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1) cnt = 3;
       if (i == B_VH_FULL || i == B_VH_FULL + 1) cnt = 4;
-      if (i == B_KC_EMPTY || i == B_KC_EMPTY + 1 || i == B_S_FREE || i == B_P_FULL || i == B_Q_FULL)
+      if (i == B_KC_EMPTY || i == B_KC_EMPTY + 1 || i == B_S_FREE || i == B_S_FREE + 1 ||
+          i == B_P_FULL || i == B_P_FULL + 1 || i == B_Q_FULL)
         cnt = 8;                                   // both softmax warpgroups
       if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = 7;   // K and V producer warps
       mbar_init(bar(i), cnt);
@@ -352,97 +440,63 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t tm_q = tmem + kColQ, tm_o = tmem + kColO, tm_p = tmem + kColP;
       const uint32_t tm_s = tmem + kColS;
-      const int64_t row_codes = D * BITS / 8;
-      const int64_t row_meta = static_cast<int64_t>(NG) * 2 * (p.meta_f16 ? 2 : 4);
-      int next_load = 0, next_s = 0, next_pv = 0;
-      bool q_ready = false;
-      long long t_idle = clock64();
-      while (next_pv < T) {
-        bool progress = false;
-        // Bulk copies of the next cached tile, as far ahead as the stage ring allows.
-        if (next_load < Tc && next_load < next_s + kStages) {
-          const int s = next_load % kStages, k = next_load / kStages;
-          if (mbar_test(bar(B_PK_EMPTY + s), (k & 1) ^ 1)) {
-            const uint32_t dst = smem_u32(smem + L.pk + s * L.stage);
-            const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(next_load) * N;
-            const uint32_t fb = bar(B_PK_FULL + s);
-            mbar_arrive_expect_tx(fb, 2 * (C::kCodes + L.meta));
-            bulk_g2s(dst, p.k_codes + row0 * row_codes, C::kCodes, fb);
-            bulk_g2s(dst + C::kCodes, static_cast<const uint8_t*>(p.k_meta) + row0 * row_meta, L.meta, fb);
-            bulk_g2s(dst + C::kCodes + L.meta, p.v_codes + row0 * row_codes, C::kCodes, fb);
-            bulk_g2s(dst + 2 * C::kCodes + L.meta,
-                     static_cast<const uint8_t*>(p.v_meta) + row0 * row_meta, L.meta, fb);
-            ++next_load;
-            progress = true;
-          }
-        }
-        if (!q_ready) q_ready = mbar_test(bar(B_Q_FULL), 0);
-        // S_j = Q K_j^T once K_j is in smem and the softmax has read S_{j-1}.
-        if (q_ready && next_s < T && mbar_test(bar(B_KH_FULL + (next_s & 1)), (next_s >> 1) & 1) &&
-            (next_s == 0 || mbar_test(bar(B_S_FREE), (next_s - 1) & 1))) {
-          const int j = next_s, sb = j & 1;
-          tc_fence_after();
-          const uint32_t kbase = smem_u32(smem + L.kt + sb * C::kTile);
-          // K tile [d/64][N keys][64], 128B swizzle, K-major: 16 channels per step (32 bytes inside
-          // the swizzle row), SBO = next 8 keys.
-          auto kdesc = [&](int ch) {
-            return smem_desc_sw128(kbase + (ch >> 6) * C::kDblk + ((ch & 63) >> 4) * 32u, 16u, 1024u);
-          };
-          if (j < Tc) {
+      const uint64_t kdesc[2] = {smem_desc_sw128(smem_u32(smem + L.kt), 16u, 1024u),
+                                 smem_desc_sw128(smem_u32(smem + L.kt + C::kTile), 16u, 1024u)};
+      const uint64_t vdesc[2] = {smem_desc_sw128(smem_u32(smem + L.vt), C::kDblk, 1024u),
+                                 smem_desc_sw128(smem_u32(smem + L.vt + C::kTile), C::kDblk, 1024u)};
+      const uint64_t adesc = smem_desc_noswz(smem_u32(ax), 128u, 256u);
+      const uint64_t bdesc[2] = {smem_desc_noswz(smem_u32(bx), 128u, 256u),
+                                 smem_desc_noswz(smem_u32(bx + C::kBx), 128u, 256u)};
+      // O += P_i V_i once the softmax wrote P_i and V_i is in smem.
+      auto issue_pv = [&](int i) -> bool {
+        const int sb = i & 1;
+        if (!mbar_wait(bar(B_P_FULL + sb), (i >> 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(bar(B_VH_FULL + sb), (i >> 1) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
+        for (int kk = 0; kk < N / 16; ++kk)   // 16 keys = two 1024-byte atoms per step
+          mma_ts(tm_o, tm_p + sb * 32u + kk * 8u, vdesc[sb] + kk * (2048u >> 4), idesc_pv,
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(bar(B_VH_EMPTY + sb));
+        tc_commit(bar(B_PV_DONE + sb));
+        return true;
+      };
+      bool ok = T > 0 && mbar_wait(bar(B_Q_FULL), 0, abort_flag, p.status);
+      if (ok) tc_fence_after();
+      // In order: S_j (once K_j is in smem and S buffer j & 1 was read), then P_{j-1}.V_{j-1}.
+      for (int j = 0; j < T && ok; ++j) {
+        const int sb = j & 1;
+        if (!mbar_wait(bar(B_KH_FULL + sb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (j >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tm_sj = tm_s + sb * 128u;
+        // K tile [d/64][N keys][64], 128B swizzle, K-major: 16 channels per step (32 bytes inside
+        // the swizzle row), SBO = next 8 keys; descriptor start addresses advance in 16-byte units.
+        auto kofs = [](int ch) { return static_cast<uint64_t>(((ch >> 6) * C::kDblk + ((ch & 63) >> 4) * 32u) >> 4); };
+        // k-steps interleaved over the accumulators (independent chains)
 #pragma unroll
-              for (int kk = 0; kk < C::G / 16; ++kk) {
-                const int ch = g * C::G + kk * 16;
-                mma_ts(tm_s + g * N, tm_q + ch / 2, kdesc(ch), idesc_s, kk > 0 ? 1u : 0u);
-              }
-          } else {
+        for (int kk = 0; kk < C::GA / 16; ++kk)
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_ts(tm_s, tm_q + kk * 8, kdesc(kk * 16), idesc_s, kk > 0 ? 1u : 0u);
+          for (int a = 0; a < C::NA; ++a) {
+            const int ch = a * C::GA + kk * 16;
+            mma_ts(tm_sj + a * N, tm_q + ch / 2, kdesc[sb] + kofs(ch), idesc_s, kk > 0 ? 1u : 0u);
           }
-          tc_commit(bar(B_KH_EMPTY + sb));
-          tc_commit(bar(B_S_FULL));
-          ++next_s;
-          progress = true;
-        }
-        // O += P_i V_i once the softmax wrote P_i and V_i is in smem.
-        if (next_pv < next_s && mbar_test(bar(B_P_FULL), next_pv & 1) &&
-            mbar_test(bar(B_VH_FULL + (next_pv & 1)), (next_pv >> 1) & 1)) {
-          const int i = next_pv, sb = i & 1;
-          tc_fence_after();
-          const uint32_t vbase = smem_u32(smem + L.vt + sb * C::kTile);
+        if (j < Tc) {
+          // zero-point and correction terms: row extras x key extras (no swizzle, K-major), into
+          // the first accumulator of each group
 #pragma unroll
-          for (int kk = 0; kk < N / 16; ++kk) {
-            // V tile [d/64][N keys][64], 128B swizzle, MN-major: 16 keys per step (two 1024-byte
-            // atoms), LBO = next 64 channels, SBO = next 8 keys.
-            const uint64_t desc = smem_desc_sw128(vbase + kk * 2048u, C::kDblk, 1024u);
-            mma_ts(tm_o, tm_p + kk * 8u, desc, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(bar(B_VH_EMPTY + sb));
-          tc_commit(bar(B_PV_DONE));
-          ++next_pv;
-          progress = true;
+          for (int g = 0; g < NG; ++g)
+            mma_ss(tm_sj + g * (C::NA / NG) * N, adesc + g * ((kBM * 32) >> 4),
+                   bdesc[sb] + g * ((N * 32) >> 4), idesc_s, 1u);
         }
-        if (progress) {
-          t_idle = clock64();
-        } else {
-          __nanosleep(32);   // leave the issue slots of this sub-partition to the other warps
-          if (*abort_flag) break;
-          if (clock64() - t_idle > kWaitLimitCycles) {
-            *abort_flag = 1;
-            atomicCAS(p.status, 0, -5);
-            break;
-          }
-        }
+        tc_commit(bar(B_KH_EMPTY + sb));
+        tc_commit(bar(B_S_FULL + sb));
+        if (j >= 1) ok = issue_pv(j - 1);
       }
+      if (ok) issue_pv(T - 1);
       // Never free tensor memory under a running MMA, never leave with copies in flight.
       tc_commit(bar(B_DRAIN));
       mbar_wait_drain(bar(B_DRAIN), 0);
-      for (int s = 0; s < kStages && s < next_load; ++s) {
-        const int last = ((next_load - 1 - s) / kStages) * kStages + s;
-        mbar_wait_drain(bar(B_PK_FULL + s), (last / kStages) & 1);
-      }
     }
     __syncwarp();
   } else if (wg == 0) {
@@ -482,22 +536,28 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
             for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
           store32<N>(kt, key, blk, v);
-          if ((blk * 32) % C::G == 0) {
+          if ((blk * 32) % C::GA == 0) {
             const int g = (blk * 32) / C::G;
-            float a = 0.f, z = 0.f, d2 = 0.f;
+            const int acc = (blk * 32) / C::GA;
+            const bool first_of_group = (blk * 32) % C::G == 0;
+            float a = 0.f, rho = 0.f, sigma = 0.f;
             if (key < valid) {
               float step, zp;
               if (p.meta_f16) load_meta<true>(kmeta, key * NG + g, step, zp);
               else load_meta<false>(kmeta, key * NG + g, step, zp);
-              a = step * p.scale_log2;
-              z = (zp - 128.f * step) * p.scale_log2;
-              d2 = step * step;
+              const float sp = step > 0.f ? step : 1.f;     // a constant group has code 0 everywhere
+              a = sp * p.scale_log2;
+              rho = zp / sp;
+              sigma = step * p.inv_scale_log2;
             }
-            float* az = reinterpret_cast<float*>(kc + (key >> 1) * NG + g);
-            az[key & 1] = a;
-            az[2 + (key & 1)] = z;
-            float* dd = reinterpret_cast<float*>(kc + (N / 2) * NG + (key >> 1) * C::NGH + (g >> 1));
-            dd[(g & 1) * 2 + (key & 1)] = d2;
+            reinterpret_cast<float*>(kc + (key >> 1) * C::NAH + (acc >> 1))[(acc & 1) * 2 + (key & 1)] = a;
+            if (!first_of_group) continue;
+            __nv_bfloat16 rh, rm, rl, sh, sm, sl;
+            split3(rho, rh, rm, rl);
+            split3(sigma, sh, sm, sl);
+            const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
+            const __nv_bfloat16 e[16] = {rh, rm, rh, sh, sm, sh, sl, sh, sm, z0, z0, z0, z0, z0, z0, z0};
+            store_extras(bx + sb * C::kBx + g * (N * 32), key, e);
           }
         }
         fence_async_smem();
@@ -521,6 +581,29 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     // ---------------------------------------------------------------- V operand tiles
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = threadIdx.x - 384;
+    // Lane 0 of the first V warp also issues the bulk copies of packed tiles, kStages - 1 ahead.
+    const bool loader = t == 0;
+    const int64_t row_codes = D * BITS / 8;
+    const int64_t row_meta = static_cast<int64_t>(NG) * 2 * (p.meta_f16 ? 2 : 4);
+    int next_load = 0;
+    auto issue_load = [&]() -> bool {
+      const int s = next_load % kStages, k = next_load / kStages;
+      if (!mbar_wait(bar(B_PK_EMPTY + s), (k & 1) ^ 1, abort_flag, p.status)) return false;
+      const uint32_t dst = smem_u32(smem + L.pk + s * L.stage);
+      const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(next_load) * N;
+      const uint32_t fb = bar(B_PK_FULL + s);
+      mbar_arrive_expect_tx(fb, 2 * (C::kCodes + L.meta));
+      bulk_g2s(dst, p.k_codes + row0 * row_codes, C::kCodes, fb);
+      bulk_g2s(dst + C::kCodes, static_cast<const uint8_t*>(p.k_meta) + row0 * row_meta, L.meta, fb);
+      bulk_g2s(dst + C::kCodes + L.meta, p.v_codes + row0 * row_codes, C::kCodes, fb);
+      bulk_g2s(dst + 2 * C::kCodes + L.meta, static_cast<const uint8_t*>(p.v_meta) + row0 * row_meta,
+               L.meta, fb);
+      ++next_load;
+      return true;
+    };
+    bool load_ok = true;
+    if (loader)
+      while (load_ok && next_load < Tc && next_load < kStages) load_ok = issue_load();
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* vt = smem + L.vt + sb * C::kTile;
@@ -561,6 +644,8 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           mbar_arrive(bar(B_VH_FULL + sb));
           mbar_arrive(bar(B_PK_EMPTY + s));
         }
+        // Tile j + kStages reuses this stage once K is done with tile j too.
+        if (loader && load_ok && next_load < Tc) load_ok = issue_load();
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
@@ -569,6 +654,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_VH_FULL + sb));
+      }
+    }
+    if (loader) {
+      for (int s = 0; s < kStages && s < next_load; ++s) {
+        const int last = ((next_load - 1 - s) / kStages) * kStages + s;
+        mbar_wait_drain(bar(B_PK_FULL + s), (last / kStages) & 1);
       }
     }
   } else {
@@ -615,6 +706,20 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         for (int k = 0; k < D / 4; ++k) qp[k] = 0u;
       }
       tmem_st<D / 4>(tmem + lane_off + kColQ + half * (D / 4), qp);
+      if (half == 0) {
+        // row extras per group: [qs_h, qs_h, qs_l, nw_h, nw_h, nw_m, nw_h, nw_l, nw_m, 0...] against
+        // the key extras [rho_h, rho_l, rho_h, sig_h, sig_m, sig_h, sig_l, sig_h, sig_m, 0...]
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          __nv_bfloat16 qh, qm, ql, nh, nm, nl;
+          split3(qs[g], qh, qm, ql);
+          split3(p.correct ? -w[g] : 0.f, nh, nm, nl);
+          const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
+          const __nv_bfloat16 e[16] = {qh, qh, qm, nh, nh, nm, nh, nl, nm, z0, z0, z0, z0, z0, z0, z0};
+          store_extras(ax + g * (kBM * 32), row, e);
+        }
+        fence_async_smem();
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -627,60 +732,47 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
 
     float m_run = -INFINITY;   // max used for the exponentials so far (log2 units), same in both halves
     float l_run = 0.f;         // this half's part of the softmax denominator
-    float2 qs2[NG], nw2[NG];   // broadcast pairs of the row's group sums and -correction weights
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      qs2[g] = make_float2(qs[g], qs[g]);
-      nw2[g] = make_float2(-w[g], -w[g]);
-    }
     const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int j = 0; j < T && ok; ++j) {
       const int sb = j & 1, n = j >> 1;
       const bool cached = j < Tc;
-      if (!warp_wait(bar(B_S_FULL), j & 1, abort_flag, p.status)) { ok = false; break; }
+      if (!warp_wait(bar(B_S_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tm_s = tmem + lane_off + kColS + kbase_h;
+      const uint32_t tm_s = tmem + lane_off + kColS + sb * 128u + kbase_h;
       float2 s2[NH / 2];         // scores of this half's key pairs (log2 units)
       int valid;                 // keys of the whole tile that count for this row
       if (cached) {
         const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
         valid = static_cast<int>(rem < N ? rem : N);
-        if (!warp_wait(bar(B_KC_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
-        const float4* az = kconst + sb * (C::kKconst / 16);
-        const float4* dd = az + (N / 2) * NG;
+        // All of this half's S columns in one batch: tcgen05.wait::ld waits for every load.
+        uint32_t r[C::NA][NH];
 #pragma unroll
-        for (int c = 0; c < NH; c += 16) {
-          uint32_t r[NG][16];
-#pragma unroll
-          for (int g = 0; g < NG; ++g) tmem_ld16(tm_s + g * N + c, r[g]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int pq = (kbase_h + c) / 2 + q;
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int gh = 0; gh < C::NGH; ++gh) {
-              const float4 d = dd[pq * C::NGH + gh];
-              acc = __ffma2_rn(make_float2(d.x, d.y), nw2[2 * gh], acc);
-              if (2 * gh + 1 < NG) acc = __ffma2_rn(make_float2(d.z, d.w), nw2[2 * gh + 1], acc);
-            }
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-              const float4 a = az[pq * NG + g];
-              acc = __ffma2_rn(make_float2(a.z, a.w), qs2[g], acc);
-              acc = __ffma2_rn(make_float2(a.x, a.y),
-                               make_float2(__uint_as_float(r[g][2 * q]), __uint_as_float(r[g][2 * q + 1])), acc);
-            }
-            s2[c / 2 + q] = acc;
-          }
-        }
+        for (int a = 0; a < C::NA; ++a) tmem_ld<NH>(tm_s + a * N, r[a]);
+        tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(B_S_FREE));
-          mbar_arrive(bar(B_KC_EMPTY + sb));
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + sb));
+        if (!warp_wait(bar(B_KC_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
+        const float4* ka = kconst + sb * (C::kKconst / 16);
+#pragma unroll
+        for (int q = 0; q < NH / 2; ++q) {
+          const int pq = kbase_h / 2 + q;
+          float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int ah = 0; ah < C::NAH; ++ah) {
+            const float4 a = ka[pq * C::NAH + ah];
+            acc = __ffma2_rn(make_float2(a.x, a.y),
+                             make_float2(__uint_as_float(r[2 * ah][2 * q]), __uint_as_float(r[2 * ah][2 * q + 1])), acc);
+            if (2 * ah + 1 < C::NA)
+              acc = __ffma2_rn(make_float2(a.z, a.w),
+                               make_float2(__uint_as_float(r[2 * ah + 1][2 * q]),
+                                           __uint_as_float(r[2 * ah + 1][2 * q + 1])), acc);
+          }
+          s2[q] = acc;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_KC_EMPTY + sb));
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         int64_t lim = cur_keys - t0;                       // keys of this tile that exist
@@ -689,18 +781,21 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           lim = c < lim ? c : lim;
         }
         valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
+        uint32_t r[C::NA][NH];
 #pragma unroll
-        for (int c = 0; c < NH; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tm_s + c, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 16; ++q)
-            s2[c / 2 + q] = __fmul2_rn(make_float2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), scale2);
-        }
+        for (int a = 0; a < C::NA; ++a) tmem_ld<NH>(tm_s + a * N, r[a]);
+        tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE));
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + sb));
+#pragma unroll
+        for (int q = 0; q < NH / 2; ++q) {
+          float2 acc = make_float2(__uint_as_float(r[0][2 * q]), __uint_as_float(r[0][2 * q + 1]));
+#pragma unroll
+          for (int a = 1; a < C::NA; ++a)
+            acc = __fadd2_rn(acc, make_float2(__uint_as_float(r[a][2 * q]), __uint_as_float(r[a][2 * q + 1])));
+          s2[q] = __fmul2_rn(acc, scale2);
+        }
       }
       if (valid < kbase_h + NH) {
 #pragma unroll
@@ -732,27 +827,30 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         m_run = m_tile;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      if (j > 0) {
-        // P and O must not be touched while the previous P.V is in flight.
-        if (!warp_wait(bar(B_PV_DONE), (j - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      // O is rescaled only after the previous P.V has finished (rare with lazy rescaling).
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if (!warp_wait(bar(B_PV_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
-          const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
-          const float2 f2 = make_float2(factor, factor);
+        const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
+        const float2 f2 = make_float2(factor, factor);
 #pragma unroll
-          for (int c = 0; c < D / 2; c += 32) {
-            uint32_t r[32];
-            tmem_ld32(tm_o + c, r);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 2; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(tm_o + c, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; k += 2) {
-              const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), f2);
-              r[k] = __float_as_uint(o2.x);
-              r[k + 1] = __float_as_uint(o2.y);
-            }
-            tmem_st32(tm_o + c, r);
+          for (int k = 0; k < 32; k += 2) {
+            const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), f2);
+            r[k] = __float_as_uint(o2.x);
+            r[k + 1] = __float_as_uint(o2.y);
           }
+          tmem_st32(tm_o + c, r);
         }
+      }
+      // P buffer j & 1 was last read by P_{j-2}.V_{j-2}.
+      if (j > 1) {
+        if (!warp_wait(bar(B_PV_DONE + sb), ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
       }
       const float2 mneg = make_float2(-m_use, -m_use);
       float2 psum = make_float2(0.f, 0.f);
@@ -764,18 +862,18 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         psum = __fadd2_rn(psum, pp);
         pk[k] = pack_bf16x2(pp.x, pp.y);
       }
-      tmem_st<NH / 2>(tmem + lane_off + kColP + kbase_h / 2, pk);
+      tmem_st<NH / 2>(tmem + lane_off + kColP + sb * 32u + kbase_h / 2, pk);
       l_run += psum.x + psum.y;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_P_FULL));
+      if (lane == 0) mbar_arrive(bar(B_P_FULL + sb));
     }
 
     // Epilogue: combine the two halves' denominators, O / l (each half writes half the columns), LSE.
     bool have_o = false;
     if (ok && T > 0) {
-      have_o = warp_wait(bar(B_PV_DONE), (T - 1) & 1, abort_flag, p.status);
+      have_o = warp_wait(bar(B_PV_DONE + ((T - 1) & 1)), ((T - 1) >> 1) & 1, abort_flag, p.status);
       tc_fence_after();
     }
     xsum[half * kBM + row] = l_run;

@@ -205,6 +205,7 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
   p.scale_log2 = sc * log2e;
   p.wcoef_log2 = sc * sc / 24.0f * log2e;
+  p.inv_scale_log2 = 1.0f / (sc * log2e);
   e = dtype == QKV_F32 ? launch_attention_f32(p, cache->d, cache->bits, static_cast<cudaStream_t>(stream))
                        : launch_attention_bf16(p, cache->d, cache->bits, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");

@@ -45,6 +45,7 @@ struct AttnParams {
   int in_f32, meta_f16;
   float scale_log2;   // score scale * log2(e)
   float wcoef_log2;   // scale^2 / 24 * log2(e): Jensen-correction coefficient in log2 units
+  float inv_scale_log2;  // 1 / (scale * log2(e))
 };
 // bf16 inputs: tcgen05 kernel. fp32 inputs: CUDA-core fp32 kernel.
 cudaError_t launch_attention_bf16(const AttnParams& p, int d, int bits, cudaStream_t stream);
