@@ -11,6 +11,7 @@ resident in HBM; L2 is flushed (a 256 MiB write) between timed steps, outside th
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -40,6 +41,69 @@ def load_peaks():
             p = json.load(f)
         return p, "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------------------------ ncu traffic
+# DRAM bytes per launch come from one ncu capture per kernel and workload, stored with a hash of
+# the kernel's sources; a stored figure is reported only while the sources still hash the same.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+CSRC = os.path.join(ROOT, "quantized_kv_cache_19_b200", "csrc")
+KERNEL_SOURCES = {
+    "corrected_attention_kernel": ["attention.cu", "qkv_common.cuh", "qkv_jensen.cuh", "qkv_internal.h"],
+    "quantize_append_kernel": ["quant_append.cu", "qkv_common.cuh", "qkv_internal.h"],
+}
+
+
+def source_hash(kernel: str) -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM read+write bytes per launch from the stored capture, or None if absent or stale."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            entry = json.load(f).get(kernel, {}).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not entry or entry.get("source_sha256") != source_hash(kernel):
+        return None
+    return entry["dram_bytes_per_launch"]
+
+
+def record_traffic(report: str, workload: str, command: str) -> None:
+    """Reads dram__bytes_{read,write}.sum of every kernel in an ncu report and stores them."""
+    import csv
+    import io
+    import subprocess
+    out = subprocess.run(["ncu", "-i", report, "--page", "raw", "--csv"], check=True,
+                         capture_output=True, text=True).stdout
+    rows = list(csv.reader(io.StringIO(out)))
+    hdr = rows[0]
+    col = {name: hdr.index(name) for name in ("Kernel Name", "dram__bytes_read.sum", "dram__bytes_write.sum")}
+    units = rows[1]
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    try:
+        with open(TRAFFIC_FILE) as f:
+            data = json.load(f)
+    except (OSError, ValueError):
+        data = {}
+    for r in rows[2:]:
+        name = r[col["Kernel Name"]].split("(")[0].split("<")[0].strip()
+        kernel = next((k for k in KERNEL_SOURCES if k in name), None)
+        if kernel is None:
+            continue
+        total = sum(float(r[col[m]].replace(",", "")) * scale[units[col[m]]]
+                    for m in ("dram__bytes_read.sum", "dram__bytes_write.sum"))
+        data.setdefault(kernel, {})[workload] = {
+            "dram_bytes_per_launch": int(round(total)), "source_sha256": source_hash(kernel),
+            "command": command}
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
 
 
 def describe(w) -> str:
@@ -264,10 +328,12 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "corrected_attention_kernel",
                      "achieved": round(achieved, 2), "peak": peak_t, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_t, 4), "peak_kind": f"{peak_kind} bf16 dense (burst)",
-                     "traffic": args.traffic, "ms_per_launch": round(ms_attn, 5),
+                     "traffic": ncu_traffic("corrected_attention_kernel", w.name),
+                     "ms_per_launch": round(ms_attn, 5),
                      "flops_per_launch": flops},
         "quant_append": {"bound": "hbm", "ms_per_launch": round(mean_qa, 5),
                          "bytes_per_launch": qa_bytes,
+                         "traffic": ncu_traffic("quantize_append_kernel", w.name),
                          "achieved_gbs": round(qa_bytes / (mean_qa * 1e-3) / 1e9, 1),
                          "peak_gbs": float(peaks["hbm_gbs"]),
                          "frac": round(qa_bytes / (mean_qa * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4)},
@@ -319,9 +385,13 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="DRAM bytes per attention launch from an ncu capture of the current kernel")
+    ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
+                    help="store the DRAM bytes per launch of an ncu report (taken on --workload) and exit")
+    ap.add_argument("--record-command", default="", help="the command line that made the report")
     args = ap.parse_args(argv)
+    if args.record_traffic:
+        record_traffic(args.record_traffic, args.workload, args.record_command)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup()
