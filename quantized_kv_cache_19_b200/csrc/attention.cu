@@ -15,32 +15,35 @@
 // sum_{c in g} q_ic^2 (so that a * w * sigma is the Jensen term b). The bracket is one tensor-core
 // accumulator per group: the codes are exact small integers in bf16 (fp32 accumulate), and the
 // two rank-1 terms ride on one extra 16-channel k-step per group whose operands are the row and
-// key values split into bf16 parts (hi+lo for rho, hi+mid+lo for the correction), which keeps
-// them to ~1e-5 of the zero-point term and ~1e-7 of b. The softmax then needs one FMA per group
+// key values split into three bf16 parts each (every product of parts whose orders add up to at
+// most two), which keeps both terms to ~2^-24 relative. The softmax then needs one FMA per group
 // per score. Rounding keys to bf16 instead would move the log-sum-exp by up to ~3e-2 on keys with
 // outlier channels. Values are dequantised to bf16 (x_hat in fp32, then rounded) for P.V.
 //
 // One CTA computes 128 packed query rows (the Hq/Hkv query heads of one KV head; row =
-// head_in_group * Lq + i) against every key of its (batch, KV head); tiles of N keys
-// (N = 64, or 32 with four groups). Four warpgroups, registers rebalanced with setmaxnreg:
+// head_in_group * Lq + i) against every key of its (batch, KV head), in tiles of N = 128 keys (64
+// with four groups), so that every MMA has N = 128 or four independent accumulators: a dependent
+// chain of 128 x 64 x 16 MMAs into one accumulator issues at a third of the tensor rate. Four
+// warpgroups, registers rebalanced with setmaxnreg:
 //   WG0      warp 0: allocates tensor memory; one thread issues, in order, S_j = Q K_j^T and then
-//            P_{j-1} V_{j-1} with precomputed descriptors (an MMA issue blocks while the tensor
-//            pipe is busy, so one lean ordered stream keeps it fed). Warps 1-3: K operand tiles (codes unpacked to bf16
-//            integers, 128-byte swizzle, 2-slot ring) and the per-key constants (a, z, step^2);
-//            for current tiles, a copy of K_cur.
+//            P_{j-1} V_{j-1} with precomputed descriptors. Warps 1-3: K operand tiles (codes
+//            unpacked to exact bf16 integers, 128-byte swizzle, two buffers); for current tiles,
+//            a copy of K_cur. Channels are stored in an operand order (k, k+8 interleaved inside
+//            each 16-channel block) that makes the unpack three operations per channel pair;
+//            Q in tensor memory and K_cur use the same order.
 //   WG1/WG2  softmax, one query row per thread, WG1 on the first half of every key tile and WG2
 //            on the second: Q row statistics and a bf16 copy of Q into TMEM; per tile read S from
 //            TMEM (releasing it at once), form the corrected scores, exchange the row max through
 //            shared memory, online softmax in base 2 with lazy rescaling of O (each half rescales
 //            half of O's columns), P (bf16) into TMEM; finally O / l and LSE.
-//   WG3      V operand tiles: dequantised to bf16; for current tiles, a copy of V_cur. One lane
-//            also issues the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point of
-//            N keys, K and V) into a 3-4 stage ring, as soon as K and V are done with a stage.
-// Tensor memory (512 columns): O [0, d), Q [128, 128 + d/2), P two buffers of N/2 at 192 and 224,
-// S two buffers of groups * N at 256 and 384 (current tiles use the first N columns of a buffer).
-// With both S and P double-buffered, the softmax of tile j+1 proceeds while P_j.V_j runs; it waits
-// for the previous P.V only to rescale O (rare: lazy rescaling) and for P.V two tiles back before
-// reusing a P buffer.
+//            The same warps then write the tile's per-key constants (scales a for the softmax,
+//            key extras for the S MMA).
+//   WG3      V operand tiles, dequantised to bf16; for current tiles, a copy of V_cur. One lane
+//            also issues the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point
+//            of N keys, K and V) into a 2-3 stage ring.
+// Tensor memory (512 columns): O [0, d), Q [128, 128 + d/2), P [192, 256), S [256, 512) (one
+// buffer of groups * N columns, or two with one group). The MMA for S_{j+1} runs while the
+// softmax works on tile j; the softmax waits for P_{j-1}.V_{j-1} before it writes P_j.
 // Every mbarrier wait is bounded; on timeout the CTA records QKV_ERR_TIMEOUT in the library's
 // device status word, drains its copies and MMAs, frees tensor memory and returns.
 #include "qkv_common.cuh"
@@ -55,10 +58,10 @@ namespace {
 constexpr int kBM = 128;                     // query rows per CTA (MMA M)
 constexpr int kThreads = 512;                 // four warpgroups
 constexpr int kRegProducer = 96, kRegSoftmax = 160;   // 2 * 96 + 2 * 160 = 512 = 4 * 128 at launch
-constexpr int kStagesMax = 4;                // packed-tile ring (INT2: 4 stages, INT4: 3)
+constexpr int kStagesMax = 3;                // packed-tile ring (INT2: 3 stages, INT4: 2)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when the max grows by more
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColQ = 128, kColP = 192, kColS = 256;   // P: 2 x 32, S: 2 x 128
+constexpr uint32_t kColO = 0, kColQ = 128, kColP = 192, kColS = 256;   // P: 64 columns, S: 256
 constexpr uint32_t kCodeMagic = 0x43004300u;  // bf16 pair (128 + c_lo, 128 + c_hi)
 
 enum {
@@ -74,23 +77,24 @@ enum {
 
 template <int D, int BITS, int NG>
 struct Cfg {
-  static constexpr int N = NG == 4 ? 32 : 64;           // keys per tile (S and P double-buffered)
-  static constexpr int kSCols = (NG == 1 ? 2 : NG) * N;  // TMEM columns of one S buffer (= 128)
+  // Keys per tile: 128, so that every MMA has N = 128 (a dependent chain of N = 64 MMAs into one
+  // accumulator issues at a third of the tensor rate; at N = 128 it runs at the full rate), or 64
+  // with four groups, whose four accumulators then hide the chain latency.
+  static constexpr int N = NG == 4 ? 64 : 128;
   static constexpr int G = D / NG;                       // channels per group
   static constexpr uint32_t kTile = N * D * 2;           // bf16 operand tile
   static constexpr uint32_t kCodes = N * D * BITS / 8;   // packed codes of one tile
-  // Score accumulators per tile: one per group, and at least two, so that consecutive MMAs of a
-  // tile go to independent accumulators (a chain into one accumulator at N = 64 runs at a third of
-  // the tensor rate). A one-group cache splits its channels over two accumulators of equal scale.
-  static constexpr int NA = NG == 1 ? 2 : NG;
-  static constexpr int GA = D / NA;                      // channels per accumulator
+  static constexpr int NA = NG;                          // score accumulators: one per group
   static constexpr int NAH = (NA + 1) / 2;               // float4s of scales per key pair
   // per-key scales a of one tile: for each key pair, NAH float4 (acc even: x,y; acc odd: z,w)
   static constexpr uint32_t kKconst = (N / 2) * NAH * 16;
   static constexpr uint32_t kAx = NG * kBM * 32;         // row extras, [g][128 rows][16] bf16
   static constexpr uint32_t kBx = NG * N * 32;           // key extras of one tile, [g][N][16] bf16
-  static constexpr int kStages = BITS == 2 ? 4 : 3;
+  static constexpr int kStages = BITS == 2 ? 3 : 2;      // packed-tile ring
   static constexpr uint32_t kDblk = N * 128;             // bytes between 64-channel blocks
+  static constexpr int kSCols = NA * N;                  // TMEM columns of one S buffer
+  static constexpr int kSB = 256 / kSCols;               // S buffers in the 256 S columns (1 or 2)
+  static constexpr int kPB = 64 / (N / 2);               // P buffers in the 64 P columns (1 or 2)
 };
 
 struct Layout {
@@ -128,36 +132,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Parks the thread in hardware until the phase completes or about `ns` nanoseconds pass.
-__device__ __forceinline__ void mbar_park(uint32_t bar, uint32_t parity, uint32_t ns) {
-  asm volatile(
-      "{\n\t.reg .pred P1;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 P1, [%0], %1, %2;\n\t}" ::"r"(bar),
-      "r"(parity), "r"(ns)
-      : "memory");
-}
-
-// Non-blocking test used by the single issuing thread of warp 0.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred P1;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, P1;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// 16 bf16x2 words (32 channels) of the codes as exact bf16 integers: (128 + code) built in the
-// mantissa, then 128 subtracted (exact).
-__device__ __forceinline__ uint32_t bf16x2_sub128(uint32_t v) {
-  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&v);
-  x = __hsub2(x, __floats2bfloat162_rn(128.f, 128.f));
-  return *reinterpret_cast<uint32_t*>(&x);
-}
-
 // Splits x into bf16 parts: x ~ hi + mid + lo.
 __device__ __forceinline__ void split3(float x, __nv_bfloat16& hi, __nv_bfloat16& mid, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
@@ -174,29 +148,46 @@ __device__ __forceinline__ void store_extras(uint8_t* tile, int row, const __nv_
   *reinterpret_cast<uint4*>(base + 128) = *reinterpret_cast<const uint4*>(&v[8]);
 }
 
+// Operand order of the channels of K (and of Q, which must match it) inside every block of 16
+// channels: position 2k holds channel k and position 2k + 1 holds channel k + 8 (k = 0..7). With
+// codes packed LSB-first, the codes of channels k and k + 8 then sit 16 bits apart in one 32-bit
+// word, and one bf16x2 operand word is a shift and a masked OR, (128 + c_k, 128 + c_{k+8}) with the
+// codes in the low mantissa bits of 128.0 (bf16 0x4300), and one exact bf16x2 subtraction of 128.
+__device__ __forceinline__ uint32_t sub128(uint32_t v) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&v);
+  x = __hsub2(x, __floats2bfloat162_rn(128.f, 128.f));
+  return *reinterpret_cast<uint32_t*>(&x);
+}
 template <int BITS>
 __device__ __forceinline__ void unpack_codes32(const uint8_t* codes, uint32_t (&out)[16]) {
   if constexpr (BITS == 2) {
     const uint2 w2 = *reinterpret_cast<const uint2*>(codes);
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {     // 16-bit halves: 8 codes, code k at bits 2k
-      const uint32_t word = h < 2 ? w2.x : w2.y;
-      const uint32_t half = (h & 1) ? (word >> 16) : (word & 0xFFFFu);
-      const uint32_t v = half | (half << 14);   // code 2p at bit 4p, code 2p+1 at bit 16+4p
+    for (int h = 0; h < 2; ++h) {     // one word = 16 codes = one channel block, code k at bits 2k
+      const uint32_t w = h ? w2.y : w2.x;
 #pragma unroll
-      for (int p = 0; p < 4; ++p) out[h * 4 + p] = bf16x2_sub128(((v >> (4 * p)) & 0x00030003u) | kCodeMagic);
+      for (int k = 0; k < 8; ++k) out[h * 8 + k] = sub128(((w >> (2 * k)) & 0x00030003u) | kCodeMagic);
     }
   } else {
     const uint4 w4 = *reinterpret_cast<const uint4*>(codes);
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {     // 16-bit halves: 4 codes, code k at bits 4k
-      const uint32_t word = h < 2 ? w4.x : h < 4 ? w4.y : h < 6 ? w4.z : w4.w;
-      const uint32_t half = (h & 1) ? (word >> 16) : (word & 0xFFFFu);
-      const uint32_t v = half | (half << 12);   // code 2p at bit 8p, code 2p+1 at bit 16+8p
+    for (int h = 0; h < 2; ++h) {     // two words = 16 codes = one channel block, code k at bits 4k
+      const uint32_t a = h ? w4.z : w4.x, b = h ? w4.w : w4.y;
+      const uint32_t lo = __byte_perm(a, b, 0x5410);   // codes 0-3 | codes 8-11 << 16
+      const uint32_t hi = __byte_perm(a, b, 0x7632);   // codes 4-7 | codes 12-15 << 16
 #pragma unroll
-      for (int p = 0; p < 2; ++p) out[h * 2 + p] = bf16x2_sub128(((v >> (8 * p)) & 0x000F000Fu) | kCodeMagic);
+      for (int k = 0; k < 4; ++k) {
+        out[h * 8 + k] = sub128(((lo >> (4 * k)) & 0x000F000Fu) | kCodeMagic);
+        out[h * 8 + 4 + k] = sub128(((hi >> (4 * k)) & 0x000F000Fu) | kCodeMagic);
+      }
     }
   }
+}
+
+// The same channel order applied to 8 bf16x2 words (16 channels, natural order) of Q or K_cur.
+__device__ __forceinline__ void permute16(const uint32_t* in, uint32_t* out) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out[k] = __byte_perm(in[k >> 1], in[4 + (k >> 1)], (k & 1) ? 0x7632 : 0x5410);
 }
 
 // Dequantises 32 channels: x_hat = zp + step * code (fp32 FMA on a float whose mantissa holds the
@@ -241,6 +232,15 @@ __device__ __forceinline__ void dequant32(const uint8_t* codes, float step, floa
   }
 }
 
+// (key, 32-channel block) of item `it` of a tile: eight consecutive items are eight consecutive
+// keys of one block, so that the 16-byte stores of a quarter-warp into a 128B-swizzled tile land
+// in eight different bank groups (keys of one block are 128 bytes apart, chunk c of key r sits at
+// chunk position c ^ (r & 7)).
+template <int D>
+__device__ __forceinline__ int item_key(int it) { return (it & 7) + ((it >> 3) / (D / 32)) * 8; }
+template <int D>
+__device__ __forceinline__ int item_blk(int it) { return (it >> 3) % (D / 32); }
+
 // Stores 32 channels (16 bf16x2) of row `key`, channel block `blk`, into a [d/64][N][64] bf16 tile
 // with the 128-byte swizzle.
 template <int N>
@@ -268,41 +268,42 @@ __device__ __forceinline__ void load_meta(const uint8_t* meta, int idx, float& s
 
 // Copies `valid` rows (of N) of bf16 [row][D] from global memory into a [D/64][N][64] swizzled tile;
 // rows beyond `valid` become zero. NT threads, kIters (key, 32-channel block) items each.
-template <int D, int N, int kIters, int NT>
+template <int D, int N, int kIters, int NT, bool kPermute>
 __device__ __forceinline__ void copy_rows(const uint4* src, uint8_t* tile, int valid, int t) {
   constexpr int kItems = N * (D / 32);
-  uint4 a[kIters][4];
+  constexpr int kBatch = 2;                  // items in flight per thread (register budget)
+#pragma unroll 1
+  for (int i0 = 0; i0 < kIters; i0 += kBatch) {
+    uint4 a[kBatch][4];
 #pragma unroll
-  for (int i = 0; i < kIters; ++i) {
-    const int it = t + NT * i, key = it / (D / 32), blk = it % (D / 32);
+    for (int i = 0; i < kBatch; ++i) {
+      const int it = t + NT * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      a[i][e] = (it < kItems && key < valid) ? src[key * (D / 8) + blk * 4 + e] : make_uint4(0u, 0u, 0u, 0u);
-  }
-#pragma unroll
-  for (int i = 0; i < kIters; ++i) {
-    const int it = t + NT * i, key = it / (D / 32), blk = it % (D / 32);
-    if (it >= kItems) break;
-    uint32_t v[16];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[4 * e] = a[i][e].x; v[4 * e + 1] = a[i][e].y; v[4 * e + 2] = a[i][e].z; v[4 * e + 3] = a[i][e].w;
+      for (int e = 0; e < 4; ++e)
+        a[i][e] = (i0 + i < kIters && it < kItems && key < valid) ? src[key * (D / 8) + blk * 4 + e]
+                                                                  : make_uint4(0u, 0u, 0u, 0u);
     }
-    store32<N>(tile, key, blk, v);
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int it = t + NT * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+      if (i0 + i >= kIters || it >= kItems) break;
+      uint32_t v[16];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[4 * e] = a[i][e].x; v[4 * e + 1] = a[i][e].y; v[4 * e + 2] = a[i][e].z; v[4 * e + 3] = a[i][e].w;
+      }
+      if (kPermute) {
+        uint32_t u[16];
+        permute16(v, u);
+        permute16(v + 8, u + 8);
+        store32<N>(tile, key, blk, u);
+      } else {
+        store32<N>(tile, key, blk, v);
+      }
+    }
   }
 }
 
-// 16 consecutive 32-bit columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
   constexpr int kItems = N * (D / 32);        // (key, 32-channel block) items of one tile
   constexpr int kItersV = kItems / 128;       // per V-producer thread (128 threads)
   constexpr int kItersK = (kItems + 95) / 96; // per K-producer thread (96 threads)
-  static_assert(kItems % 128 == 0, "tile items must split evenly over a warpgroup");
+  static_assert(kItems % 128 == 0 && kItersV % 2 == 0, "tile items must split evenly over a warpgroup");
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // 1024-byte alignment (128B-swizzle atoms) by offsetting the shared array itself, so that the
   // compiler keeps every access in the shared address space.
@@ -449,47 +450,46 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
                                  smem_desc_noswz(smem_u32(bx + C::kBx), 128u, 256u)};
       // O += P_i V_i once the softmax wrote P_i and V_i is in smem.
       auto issue_pv = [&](int i) -> bool {
-        const int sb = i & 1;
-        if (!mbar_wait(bar(B_P_FULL + sb), (i >> 1) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(bar(B_VH_FULL + sb), (i >> 1) & 1, abort_flag, p.status)) return false;
+        const int vb = i & 1, pb = i % C::kPB;
+        if (!mbar_wait(bar(B_P_FULL + pb), (i / C::kPB) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(bar(B_VH_FULL + vb), (i >> 1) & 1, abort_flag, p.status)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk)   // 16 keys = two 1024-byte atoms per step
-          mma_ts(tm_o, tm_p + sb * 32u + kk * 8u, vdesc[sb] + kk * (2048u >> 4), idesc_pv,
+          mma_ts(tm_o, tm_p + pb * (N / 2) + kk * 8u, vdesc[vb] + kk * (2048u >> 4), idesc_pv,
                  (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(B_VH_EMPTY + sb));
-        tc_commit(bar(B_PV_DONE + sb));
+        tc_commit(bar(B_VH_EMPTY + vb));
+        tc_commit(bar(B_PV_DONE + pb));
         return true;
       };
       bool ok = T > 0 && mbar_wait(bar(B_Q_FULL), 0, abort_flag, p.status);
       if (ok) tc_fence_after();
-      // In order: S_j (once K_j is in smem and S buffer j & 1 was read), then P_{j-1}.V_{j-1}.
+      // In order: S_j (once K_j is in smem and its S buffer was read by the softmax), then
+      // P_{j-1}.V_{j-1}.
       for (int j = 0; j < T && ok; ++j) {
-        const int sb = j & 1;
-        if (!mbar_wait(bar(B_KH_FULL + sb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        const int kb = j & 1, sb = j % C::kSB;
+        if (!mbar_wait(bar(B_KH_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (j >= C::kSB && !mbar_wait(bar(B_S_FREE + sb), ((j - C::kSB) / C::kSB) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t tm_sj = tm_s + sb * 128u;
+        const uint32_t tm_sj = tm_s + sb * C::kSCols;
         // K tile [d/64][N keys][64], 128B swizzle, K-major: 16 channels per step (32 bytes inside
         // the swizzle row), SBO = next 8 keys; descriptor start addresses advance in 16-byte units.
         auto kofs = [](int ch) { return static_cast<uint64_t>(((ch >> 6) * C::kDblk + ((ch & 63) >> 4) * 32u) >> 4); };
-        // k-steps interleaved over the accumulators (independent chains)
+        // k-steps interleaved over the group accumulators (independent chains)
 #pragma unroll
-        for (int kk = 0; kk < C::GA / 16; ++kk)
+        for (int kk = 0; kk < C::G / 16; ++kk)
 #pragma unroll
-          for (int a = 0; a < C::NA; ++a) {
-            const int ch = a * C::GA + kk * 16;
-            mma_ts(tm_sj + a * N, tm_q + ch / 2, kdesc[sb] + kofs(ch), idesc_s, kk > 0 ? 1u : 0u);
+          for (int g = 0; g < NG; ++g) {
+            const int ch = g * C::G + kk * 16;
+            mma_ts(tm_sj + g * N, tm_q + ch / 2, kdesc[kb] + kofs(ch), idesc_s, kk > 0 ? 1u : 0u);
           }
         if (j < Tc) {
-          // zero-point and correction terms: row extras x key extras (no swizzle, K-major), into
-          // the first accumulator of each group
+          // zero-point and correction terms: row extras x key extras (no swizzle, K-major)
 #pragma unroll
           for (int g = 0; g < NG; ++g)
-            mma_ss(tm_sj + g * (C::NA / NG) * N, adesc + g * ((kBM * 32) >> 4),
-                   bdesc[sb] + g * ((N * 32) >> 4), idesc_s, 1u);
+            mma_ss(tm_sj + g * N, adesc + g * ((kBM * 32) >> 4), bdesc[kb] + g * ((N * 32) >> 4), idesc_s, 1u);
         }
-        tc_commit(bar(B_KH_EMPTY + sb));
+        tc_commit(bar(B_KH_EMPTY + kb));
         tc_commit(bar(B_S_FULL + sb));
         if (j >= 1) ok = issue_pv(j - 1);
       }
@@ -512,53 +512,61 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
         const int valid = static_cast<int>(rem < N ? rem : N);
         const uint8_t* kcodes = smem + L.pk + s * L.stage;
-        const uint8_t* kmeta = kcodes + C::kCodes;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
-        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
-        float4* kc = kconst + sb * (C::kKconst / 16);
         using CodeVec = typename std::conditional<BITS == 2, uint2, uint4>::type;
-        CodeVec cv[kItersK];
+        // Two items per iteration, the loop itself not unrolled: the code of all four roles has
+        // to share the instruction caches of each SM sub-partition.
+#pragma unroll 1
+        for (int i0 = 0; i0 < kItersK; i0 += 2) {
+          CodeVec cv[2];
 #pragma unroll
-        for (int i = 0; i < kItersK; ++i) {
-          const int it = t + 96 * i, key = it / (D / 32), blk = it % (D / 32);
-          if (it < kItems)
-            cv[i] = *reinterpret_cast<const CodeVec*>(kcodes + key * (D * BITS / 8) + blk * (4 * BITS));
-        }
-#pragma unroll
-        for (int i = 0; i < kItersK; ++i) {
-          const int it = t + 96 * i, key = it / (D / 32), blk = it % (D / 32);
-          if (it >= kItems) break;
-          uint32_t v[16];
-          if (key < valid) {
-            unpack_codes32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0u;
+          for (int i = 0; i < 2; ++i) {
+            const int it = t + 96 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+            if (it < kItems)
+              cv[i] = *reinterpret_cast<const CodeVec*>(kcodes + key * (D * BITS / 8) + blk * (4 * BITS));
           }
-          store32<N>(kt, key, blk, v);
-          if ((blk * 32) % C::GA == 0) {
-            const int g = (blk * 32) / C::G;
-            const int acc = (blk * 32) / C::GA;
-            const bool first_of_group = (blk * 32) % C::G == 0;
-            float a = 0.f, rho = 0.f, sigma = 0.f;
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int it = t + 96 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+            if (it >= kItems) break;
+            uint32_t v[16];
             if (key < valid) {
-              float step, zp;
-              if (p.meta_f16) load_meta<true>(kmeta, key * NG + g, step, zp);
-              else load_meta<false>(kmeta, key * NG + g, step, zp);
-              const float sp = step > 0.f ? step : 1.f;     // a constant group has code 0 everywhere
-              a = sp * p.scale_log2;
-              rho = zp / sp;
-              sigma = step * p.inv_scale_log2;
+              unpack_codes32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), v);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0u;
             }
-            reinterpret_cast<float*>(kc + (key >> 1) * C::NAH + (acc >> 1))[(acc & 1) * 2 + (key & 1)] = a;
-            if (!first_of_group) continue;
-            __nv_bfloat16 rh, rm, rl, sh, sm, sl;
-            split3(rho, rh, rm, rl);
-            split3(sigma, sh, sm, sl);
-            const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
-            const __nv_bfloat16 e[16] = {rh, rm, rh, sh, sm, sh, sl, sh, sm, z0, z0, z0, z0, z0, z0, z0};
-            store_extras(bx + sb * C::kBx + g * (N * 32), key, e);
+            store32<N>(kt, key, blk, v);
           }
+        }
+        // Per-key constants of the tile: scales a for the softmax (once it has read the previous
+        // ones from this buffer) and the key extras of the S MMA.
+        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+        const uint8_t* kmeta = kcodes + C::kCodes;
+        float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
+        constexpr int kItersC = (N * NG + 95) / 96;
+#pragma unroll
+        for (int i = 0; i < kItersC; ++i) {
+          const int e = t + 96 * i;
+          if (e >= N * NG) break;
+          const int key = e / NG, g = e % NG;
+          float a = 0.f, rho = 0.f, sigma = 0.f;
+          if (key < valid) {
+            float step, zp;
+            if (p.meta_f16) load_meta<true>(kmeta, key * NG + g, step, zp);
+            else load_meta<false>(kmeta, key * NG + g, step, zp);
+            const float sp = step > 0.f ? step : 1.f;     // a constant group has code 0 everywhere
+            a = sp * p.scale_log2;
+            rho = zp / sp;
+            sigma = step * p.inv_scale_log2;
+          }
+          kc[((key >> 1) * C::NAH + (g >> 1)) * 4 + (g & 1) * 2 + (key & 1)] = a;
+          __nv_bfloat16 rh, rm, rl, sh, sm, sl;
+          split3(rho, rh, rm, rl);
+          split3(sigma, sh, sm, sl);
+          const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
+          const __nv_bfloat16 x16[16] = {rh, rm, rh, rl, rm, rh, sh, sm, sh, sl, sh, sm, z0, z0, z0, z0};
+          store_extras(bx + sb * C::kBx + g * (N * 32), key, x16);
         }
         fence_async_smem();
         __syncwarp();
@@ -571,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
         const uint4* src = reinterpret_cast<const uint4*>(p.K_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
-        copy_rows<D, N, kItersK, 96>(src, kt, valid, t);
+        copy_rows<D, N, kItersK, 96, true>(src, kt, valid, t);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_KH_FULL + sb));
@@ -616,27 +624,31 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const uint8_t* vmeta = vcodes + C::kCodes;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
         using CodeVec = typename std::conditional<BITS == 2, uint2, uint4>::type;
-        CodeVec cv[kItersV];
-        float st[kItersV], zp[kItersV];
+        constexpr int kBatch = 2;                 // items per iteration; the loop is not unrolled
+#pragma unroll 1
+        for (int i0 = 0; i0 < kItersV; i0 += kBatch) {
+          CodeVec cv[kBatch];
+          float st[kBatch], zp[kBatch];
 #pragma unroll
-        for (int i = 0; i < kItersV; ++i) {
-          const int it = t + 128 * i, key = it / (D / 32), blk = it % (D / 32);
-          const int g = (blk * 32) / C::G;
-          cv[i] = *reinterpret_cast<const CodeVec*>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS));
-          if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, st[i], zp[i]);
-          else load_meta<false>(vmeta, key * NG + g, st[i], zp[i]);
-        }
-#pragma unroll
-        for (int i = 0; i < kItersV; ++i) {
-          const int it = t + 128 * i, key = it / (D / 32), blk = it % (D / 32);
-          uint32_t v[16];
-          if (key < valid) {
-            dequant32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), st[i], zp[i], v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0u;
+          for (int i = 0; i < kBatch; ++i) {
+            const int it = t + 128 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+            const int g = (blk * 32) / C::G;
+            cv[i] = *reinterpret_cast<const CodeVec*>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS));
+            if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, st[i], zp[i]);
+            else load_meta<false>(vmeta, key * NG + g, st[i], zp[i]);
           }
-          store32<N>(vt, key, blk, v);
+#pragma unroll
+          for (int i = 0; i < kBatch; ++i) {
+            const int it = t + 128 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+            uint32_t v[16];
+            if (key < valid) {
+              dequant32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), st[i], zp[i], v);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0u;
+            }
+            store32<N>(vt, key, blk, v);
+          }
         }
         fence_async_smem();
         __syncwarp();
@@ -650,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
         const uint4* src = reinterpret_cast<const uint4*>(p.V_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
-        copy_rows<D, N, kItersV, 128>(src, vt, valid, t);
+        copy_rows<D, N, kItersV, 128, false>(src, vt, valid, t);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_VH_FULL + sb));
@@ -697,9 +709,11 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
             if (g == (c8 * 8) / C::G) qs[g] += acc;
         }
 #pragma unroll
-        for (int c8 = 0; c8 < D / 16; ++c8) {
-          const uint4 u = reinterpret_cast<const uint4*>(qrow)[half * (D / 16) + c8];
-          qp[4 * c8] = u.x; qp[4 * c8 + 1] = u.y; qp[4 * c8 + 2] = u.z; qp[4 * c8 + 3] = u.w;
+        for (int c8 = 0; c8 < D / 16; c8 += 2) {   // 16 channels at a time, in operand order
+          const uint4 u0 = reinterpret_cast<const uint4*>(qrow)[half * (D / 16) + c8];
+          const uint4 u1 = reinterpret_cast<const uint4*>(qrow)[half * (D / 16) + c8 + 1];
+          const uint32_t nat[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          permute16(nat, qp + 4 * c8);
         }
       } else {
 #pragma unroll
@@ -707,15 +721,16 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       }
       tmem_st<D / 4>(tmem + lane_off + kColQ + half * (D / 4), qp);
       if (half == 0) {
-        // row extras per group: [qs_h, qs_h, qs_l, nw_h, nw_h, nw_m, nw_h, nw_l, nw_m, 0...] against
-        // the key extras [rho_h, rho_l, rho_h, sig_h, sig_m, sig_h, sig_l, sig_h, sig_m, 0...]
+        // row extras per group [qs_h, qs_h, qs_m, qs_h, qs_m, qs_l, nw_h, nw_h, nw_m, nw_h, nw_l, nw_m, 0..]
+        // against the key extras [rho_h, rho_m, rho_h, rho_l, rho_m, rho_h, sig_h, sig_m, sig_h, sig_l,
+        // sig_h, sig_m, 0..]: every product of parts whose orders add up to at most two.
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
           __nv_bfloat16 qh, qm, ql, nh, nm, nl;
           split3(qs[g], qh, qm, ql);
           split3(p.correct ? -w[g] : 0.f, nh, nm, nl);
           const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
-          const __nv_bfloat16 e[16] = {qh, qh, qm, nh, nh, nm, nh, nl, nm, z0, z0, z0, z0, z0, z0, z0};
+          const __nv_bfloat16 e[16] = {qh, qh, qm, qh, qm, ql, nh, nh, nm, nh, nl, nm, z0, z0, z0, z0};
           store_extras(ax + g * (kBM * 32), row, e);
         }
         fence_async_smem();
@@ -734,45 +749,51 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     float l_run = 0.f;         // this half's part of the softmax denominator
     const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
+    // S columns are read in chunks of kCK keys (NA * kCK registers); tcgen05.wait::ld waits for
+    // every load of a chunk.
+    constexpr int kCK = C::NA == 1 ? 32 : 64 / C::NA;
     for (int j = 0; j < T && ok; ++j) {
-      const int sb = j & 1, n = j >> 1;
+      const int kb = j & 1, sbuf = j % C::kSB, pb = j % C::kPB;
       const bool cached = j < Tc;
-      if (!warp_wait(bar(B_S_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
+      if (!warp_wait(bar(B_S_FULL + sbuf), (j / C::kSB) & 1, abort_flag, p.status)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tm_s = tmem + lane_off + kColS + sb * 128u + kbase_h;
+      const uint32_t tm_s = tmem + lane_off + kColS + sbuf * C::kSCols + kbase_h;
       float2 s2[NH / 2];         // scores of this half's key pairs (log2 units)
       int valid;                 // keys of the whole tile that count for this row
       if (cached) {
         const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
         valid = static_cast<int>(rem < N ? rem : N);
-        // All of this half's S columns in one batch: tcgen05.wait::ld waits for every load.
-        uint32_t r[C::NA][NH];
+        if (!warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        const float4* ka = kconst + kb * (C::kKconst / 16);
 #pragma unroll
-        for (int a = 0; a < C::NA; ++a) tmem_ld<NH>(tm_s + a * N, r[a]);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < NH; c0 += kCK) {
+          uint32_t r[C::NA][kCK];
+#pragma unroll
+          for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < kCK / 2; ++q) {
+            const int pq = (kbase_h + c0) / 2 + q;
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int ah = 0; ah < C::NAH; ++ah) {
+              const float4 a = ka[pq * C::NAH + ah];
+              acc = __ffma2_rn(make_float2(a.x, a.y),
+                               make_float2(__uint_as_float(r[2 * ah][2 * q]), __uint_as_float(r[2 * ah][2 * q + 1])), acc);
+              if (2 * ah + 1 < C::NA)
+                acc = __ffma2_rn(make_float2(a.z, a.w),
+                                 make_float2(__uint_as_float(r[2 * ah + 1][2 * q]),
+                                             __uint_as_float(r[2 * ah + 1][2 * q + 1])), acc);
+            }
+            s2[c0 / 2 + q] = acc;
+          }
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + sb));
-        if (!warp_wait(bar(B_KC_FULL + sb), n & 1, abort_flag, p.status)) { ok = false; break; }
-        const float4* ka = kconst + sb * (C::kKconst / 16);
-#pragma unroll
-        for (int q = 0; q < NH / 2; ++q) {
-          const int pq = kbase_h / 2 + q;
-          float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int ah = 0; ah < C::NAH; ++ah) {
-            const float4 a = ka[pq * C::NAH + ah];
-            acc = __ffma2_rn(make_float2(a.x, a.y),
-                             make_float2(__uint_as_float(r[2 * ah][2 * q]), __uint_as_float(r[2 * ah][2 * q + 1])), acc);
-            if (2 * ah + 1 < C::NA)
-              acc = __ffma2_rn(make_float2(a.z, a.w),
-                               make_float2(__uint_as_float(r[2 * ah + 1][2 * q]),
-                                           __uint_as_float(r[2 * ah + 1][2 * q + 1])), acc);
-          }
-          s2[q] = acc;
+        if (lane == 0) {
+          mbar_arrive(bar(B_S_FREE + sbuf));
+          mbar_arrive(bar(B_KC_EMPTY + kb));
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_KC_EMPTY + sb));
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         int64_t lim = cur_keys - t0;                       // keys of this tile that exist
@@ -781,21 +802,24 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           lim = c < lim ? c : lim;
         }
         valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
-        uint32_t r[C::NA][NH];
 #pragma unroll
-        for (int a = 0; a < C::NA; ++a) tmem_ld<NH>(tm_s + a * N, r[a]);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < NH; c0 += kCK) {
+          uint32_t r[C::NA][kCK];
+#pragma unroll
+          for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < kCK / 2; ++q) {
+            float2 acc = make_float2(__uint_as_float(r[0][2 * q]), __uint_as_float(r[0][2 * q + 1]));
+#pragma unroll
+            for (int a = 1; a < C::NA; ++a)
+              acc = __fadd2_rn(acc, make_float2(__uint_as_float(r[a][2 * q]), __uint_as_float(r[a][2 * q + 1])));
+            s2[c0 / 2 + q] = __fmul2_rn(acc, scale2);
+          }
+        }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + sb));
-#pragma unroll
-        for (int q = 0; q < NH / 2; ++q) {
-          float2 acc = make_float2(__uint_as_float(r[0][2 * q]), __uint_as_float(r[0][2 * q + 1]));
-#pragma unroll
-          for (int a = 1; a < C::NA; ++a)
-            acc = __fadd2_rn(acc, make_float2(__uint_as_float(r[a][2 * q]), __uint_as_float(r[a][2 * q + 1])));
-          s2[q] = __fmul2_rn(acc, scale2);
-        }
+        if (lane == 0) mbar_arrive(bar(B_S_FREE + sbuf));
       }
       if (valid < kbase_h + NH) {
 #pragma unroll
@@ -829,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       // O is rescaled only after the previous P.V has finished (rare with lazy rescaling).
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        if (!warp_wait(bar(B_PV_DONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (!warp_wait(bar(B_PV_DONE + (j - 1) % C::kPB), ((j - 1) / C::kPB) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
         const float2 f2 = make_float2(factor, factor);
@@ -847,9 +871,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           tmem_st32(tm_o + c, r);
         }
       }
-      // P buffer j & 1 was last read by P_{j-2}.V_{j-2}.
-      if (j > 1) {
-        if (!warp_wait(bar(B_PV_DONE + sb), ((j - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      // P buffer pb was last read by P_{j-kPB}.V_{j-kPB}.
+      if (j >= C::kPB) {
+        if (!warp_wait(bar(B_PV_DONE + pb), ((j - C::kPB) / C::kPB) & 1, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
       }
       const float2 mneg = make_float2(-m_use, -m_use);
@@ -862,18 +886,18 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         psum = __fadd2_rn(psum, pp);
         pk[k] = pack_bf16x2(pp.x, pp.y);
       }
-      tmem_st<NH / 2>(tmem + lane_off + kColP + sb * 32u + kbase_h / 2, pk);
+      tmem_st<NH / 2>(tmem + lane_off + kColP + pb * (N / 2) + kbase_h / 2, pk);
       l_run += psum.x + psum.y;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_P_FULL + sb));
+      if (lane == 0) mbar_arrive(bar(B_P_FULL + pb));
     }
 
     // Epilogue: combine the two halves' denominators, O / l (each half writes half the columns), LSE.
     bool have_o = false;
     if (ok && T > 0) {
-      have_o = warp_wait(bar(B_PV_DONE + ((T - 1) & 1)), ((T - 1) >> 1) & 1, abort_flag, p.status);
+      have_o = warp_wait(bar(B_PV_DONE + (T - 1) % C::kPB), ((T - 1) / C::kPB) & 1, abort_flag, p.status);
       tc_fence_after();
     }
     xsum[half * kBM + row] = l_run;

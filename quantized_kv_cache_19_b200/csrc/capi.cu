@@ -136,7 +136,7 @@ QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const voi
   p.K = K; p.V = V;
   p.k_codes = cache->k_codes; p.v_codes = cache->v_codes;
   p.k_meta = cache->k_meta; p.v_meta = cache->v_meta;
-  p.rows = static_cast<int64_t>(cache->B) * cache->H_kv * L_new;
+  p.BH = static_cast<int64_t>(cache->B) * cache->H_kv;
   p.L_new = L_new;
   p.capacity = cache->capacity;
   p.start = cache->length;

@@ -17,7 +17,7 @@ struct QuantAppendParams {
   uint8_t* v_codes;
   void* k_meta;
   void* v_meta;
-  int64_t rows;      // B * H_kv * L_new token-head rows per tensor
+  int64_t BH;        // B * H_kv
   int64_t L_new;
   int64_t capacity;
   int64_t start;

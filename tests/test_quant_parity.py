@@ -91,3 +91,32 @@ def test_other_codecs(bits, group, meta, dtype):
     torch.cuda.synchronize()
     idx = np.stack(np.meshgrid(np.arange(1), np.arange(3), np.arange(257), indexing="ij"), -1).reshape(-1, 3)
     _compare_rows(w, cache, x["K_src"], x["V_src"], idx)
+
+
+@pytest.mark.parametrize("bits,meta,d,group", [(2, "f32", 128, 64), (4, "f32", 64, 32),
+                                                (2, "f16", 64, 64), (4, "f16", 128, 128)])
+def test_exact_ties_round_to_even(bits, meta, d, group):
+    """Groups laid on a half-step grid, so that (x - min) / step is exactly k + 1/2 for about half of
+    the channels; rint must pick the even code there (oracle: round half to even)."""
+    levels = (1 << bits) - 1
+    rows, n_g = 96, d // group
+    rng = np.random.default_rng(11 + bits)
+    h = rng.integers(0, 2 * levels + 1, size=(rows, n_g, group))
+    h[:, :, 0], h[:, :, 1] = 0, 2 * levels                      # min and max present in every group
+    for r in range(rows):                                       # shuffle each group's channels
+        for g in range(n_g):
+            rng.shuffle(h[r, g])
+    base = rng.integers(-8, 8, size=(rows, n_g, 1)) * 0.25      # zero-point, exact in bf16
+    scale = 2.0 ** rng.integers(-3, 1, size=(rows, n_g, 1))     # step: a power of two
+    x = (base + scale * h / 2).reshape(1, 1, rows, d)
+    K = torch.tensor(x, dtype=torch.bfloat16, device="cuda")
+    assert torch.equal(K.float().cpu(), torch.tensor(x, dtype=torch.float32))   # exact in bf16
+    V = (-K).contiguous()
+    w = WORKLOADS["bf16_int2"].with_(Hq=1, Hkv=1, d=d, Lc=rows, bits=bits, group=group, meta=meta)
+    cache = api.KVCache(1, 1, d, bits, group, 128, meta)
+    api.kv_quantize_append(cache, K, V)
+    torch.cuda.synchronize()
+    ties = (np.asarray(h) % 2 == 1).mean()
+    assert ties > 0.3
+    idx = np.stack([np.zeros(rows, int), np.zeros(rows, int), np.arange(rows)], -1)
+    _compare_rows(w, cache, K, V, idx)
