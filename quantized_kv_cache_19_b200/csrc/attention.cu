@@ -142,10 +142,13 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16& hi, __nv_bfloat16
 
 // 16 bf16 channels of one row of an extras tile in the no-swizzle K-major core-matrix layout
 // [row / 8][2 halves][row % 8][8].
-__device__ __forceinline__ void store_extras(uint8_t* tile, int row, const __nv_bfloat16 (&v)[16]) {
+__device__ __forceinline__ void store_extras(uint8_t* tile, int row, uint4 lo8, uint4 hi8) {
   uint8_t* base = tile + (row >> 3) * 256 + (row & 7) * 16;
-  *reinterpret_cast<uint4*>(base) = *reinterpret_cast<const uint4*>(&v[0]);
-  *reinterpret_cast<uint4*>(base + 128) = *reinterpret_cast<const uint4*>(&v[8]);
+  *reinterpret_cast<uint4*>(base) = lo8;
+  *reinterpret_cast<uint4*>(base + 128) = hi8;
+}
+__device__ __forceinline__ uint32_t bf_pair(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
 }
 
 // Operand order of the channels of K (and of Q, which must match it) inside every block of 16
@@ -564,9 +567,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           __nv_bfloat16 rh, rm, rl, sh, sm, sl;
           split3(rho, rh, rm, rl);
           split3(sigma, sh, sm, sl);
-          const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
-          const __nv_bfloat16 x16[16] = {rh, rm, rh, rl, rm, rh, sh, sm, sh, sl, sh, sm, z0, z0, z0, z0};
-          store_extras(bx + sb * C::kBx + g * (N * 32), key, x16);
+          // [rho_h, rho_m, rho_h, rho_l, rho_m, rho_h, sig_h, sig_m, sig_h, sig_l, sig_h, sig_m, 0, 0, 0, 0]
+          store_extras(bx + sb * C::kBx + g * (N * 32), key,
+                       make_uint4(bf_pair(rh, rm), bf_pair(rh, rl), bf_pair(rm, rh), bf_pair(sh, sm)),
+                       make_uint4(bf_pair(sh, sl), bf_pair(sh, sm), 0u, 0u));
         }
         fence_async_smem();
         __syncwarp();
@@ -581,8 +585,17 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const uint4* src = reinterpret_cast<const uint4*>(p.K_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
         copy_rows<D, N, kItersK, 96, true>(src, kt, valid, t);
         fence_async_smem();
+        // Scales of the current tile: the plain score scale for every key and group, so that the
+        // softmax forms every tile's scores the same way.
+        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+        float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
+#pragma unroll 1
+        for (int e = t; e < static_cast<int>(C::kKconst / 4); e += 96) kc[e] = p.scale_log2;
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_KH_FULL + sb));
+        if (lane == 0) {
+          mbar_arrive(bar(B_KH_FULL + sb));
+          mbar_arrive(bar(B_KC_FULL + sb));
+        }
       }
     }
   } else if (wg == 3) {
@@ -729,9 +742,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           __nv_bfloat16 qh, qm, ql, nh, nm, nl;
           split3(qs[g], qh, qm, ql);
           split3(p.correct ? -w[g] : 0.f, nh, nm, nl);
-          const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
-          const __nv_bfloat16 e[16] = {qh, qh, qm, qh, qm, ql, nh, nh, nm, nh, nl, nm, z0, z0, z0, z0};
-          store_extras(ax + g * (kBM * 32), row, e);
+          store_extras(ax + g * (kBM * 32), row,
+                       make_uint4(bf_pair(qh, qh), bf_pair(qm, qh), bf_pair(qm, ql), bf_pair(nh, nh)),
+                       make_uint4(bf_pair(nm, nh), bf_pair(nl, nm), 0u, 0u));
         }
         fence_async_smem();
       }
@@ -763,37 +776,6 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       if (cached) {
         const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
         valid = static_cast<int>(rem < N ? rem : N);
-        if (!warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        const float4* ka = kconst + kb * (C::kKconst / 16);
-#pragma unroll
-        for (int c0 = 0; c0 < NH; c0 += kCK) {
-          uint32_t r[C::NA][kCK];
-#pragma unroll
-          for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < kCK / 2; ++q) {
-            const int pq = (kbase_h + c0) / 2 + q;
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int ah = 0; ah < C::NAH; ++ah) {
-              const float4 a = ka[pq * C::NAH + ah];
-              acc = __ffma2_rn(make_float2(a.x, a.y),
-                               make_float2(__uint_as_float(r[2 * ah][2 * q]), __uint_as_float(r[2 * ah][2 * q + 1])), acc);
-              if (2 * ah + 1 < C::NA)
-                acc = __ffma2_rn(make_float2(a.z, a.w),
-                                 make_float2(__uint_as_float(r[2 * ah + 1][2 * q]),
-                                             __uint_as_float(r[2 * ah + 1][2 * q + 1])), acc);
-            }
-            s2[c0 / 2 + q] = acc;
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(B_S_FREE + sbuf));
-          mbar_arrive(bar(B_KC_EMPTY + kb));
-        }
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         int64_t lim = cur_keys - t0;                       // keys of this tile that exist
@@ -802,24 +784,38 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           lim = c < lim ? c : lim;
         }
         valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
+      }
+      if (!warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      // s = sum_g a_g * S_g: per-key group scales for cached tiles, the score scale for current ones.
+      const float4* ka = kconst + kb * (C::kKconst / 16);
 #pragma unroll
-        for (int c0 = 0; c0 < NH; c0 += kCK) {
-          uint32_t r[C::NA][kCK];
+      for (int c0 = 0; c0 < NH; c0 += kCK) {
+        uint32_t r[C::NA][kCK];
 #pragma unroll
-          for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
-          tmem_wait_ld();
+        for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < kCK / 2; ++q) {
-            float2 acc = make_float2(__uint_as_float(r[0][2 * q]), __uint_as_float(r[0][2 * q + 1]));
+        for (int q = 0; q < kCK / 2; ++q) {
+          const int pq = (kbase_h + c0) / 2 + q;
+          float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int a = 1; a < C::NA; ++a)
-              acc = __fadd2_rn(acc, make_float2(__uint_as_float(r[a][2 * q]), __uint_as_float(r[a][2 * q + 1])));
-            s2[c0 / 2 + q] = __fmul2_rn(acc, scale2);
+          for (int ah = 0; ah < C::NAH; ++ah) {
+            const float4 a = ka[pq * C::NAH + ah];
+            acc = __ffma2_rn(make_float2(a.x, a.y),
+                             make_float2(__uint_as_float(r[2 * ah][2 * q]), __uint_as_float(r[2 * ah][2 * q + 1])), acc);
+            if (2 * ah + 1 < C::NA)
+              acc = __ffma2_rn(make_float2(a.z, a.w),
+                               make_float2(__uint_as_float(r[2 * ah + 1][2 * q]),
+                                           __uint_as_float(r[2 * ah + 1][2 * q + 1])), acc);
           }
+          s2[c0 / 2 + q] = acc;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_FREE + sbuf));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(B_S_FREE + sbuf));
+        mbar_arrive(bar(B_KC_EMPTY + kb));
       }
       if (valid < kbase_h + NH) {
 #pragma unroll
@@ -857,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         tc_fence_after();
         const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
         const float2 f2 = make_float2(factor, factor);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < D / 2; c += 32) {
           uint32_t r[32];
           tmem_ld32(tm_o + c, r);
