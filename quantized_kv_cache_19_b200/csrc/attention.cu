@@ -23,21 +23,20 @@
 // One CTA computes 128 packed query rows (the Hq/Hkv query heads of one KV head; row =
 // head_in_group * Lq + i) against every key of its (batch, KV head), in tiles of N = 128 keys (64
 // with four groups), so that every MMA has N = 128 or four independent accumulators: a dependent
-// chain of 128 x 64 x 16 MMAs into one accumulator issues at a third of the tensor rate. Four
+// chain of 128 x 64 x 16 MMAs into one accumulator issues at a third of the tensor rate. Five
 // warpgroups, registers rebalanced with setmaxnreg:
 //   WG0      warp 0: allocates tensor memory; one thread issues, in order, S_j = Q K_j^T and then
-//            P_{j-1} V_{j-1} with precomputed descriptors. Warps 1-3: K operand tiles (codes
-//            unpacked to exact bf16 integers, 128-byte swizzle, two buffers); for current tiles,
-//            a copy of K_cur. Channels are stored in an operand order (k, k+8 interleaved inside
-//            each 16-channel block) that makes the unpack three operations per channel pair;
-//            Q in tensor memory and K_cur use the same order.
+//            P_{j-1} V_{j-1} with precomputed descriptors.
+//   WG0 warps 1-3 and WG4: K operand tiles (codes unpacked to exact bf16 integers, 128-byte
+//            swizzle, two buffers) and the tile's per-key constants (scales a for the softmax, key
+//            extras for the S MMA); for current tiles, a copy of K_cur. Channels are stored in an
+//            operand order (k, k+8 interleaved inside each 16-channel block) that makes the unpack
+//            three operations per channel pair; Q in tensor memory and K_cur use the same order.
 //   WG1/WG2  softmax, one query row per thread, WG1 on the first half of every key tile and WG2
 //            on the second: Q row statistics and a bf16 copy of Q into TMEM; per tile read S from
 //            TMEM (releasing it at once), form the corrected scores, exchange the row max through
 //            shared memory, online softmax in base 2 with lazy rescaling of O (each half rescales
 //            half of O's columns), P (bf16) into TMEM; finally O / l and LSE.
-//            The same warps then write the tile's per-key constants (scales a for the softmax,
-//            key extras for the S MMA).
 //   WG3      V operand tiles, dequantised to bf16; for current tiles, a copy of V_cur. One lane
 //            also issues the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point
 //            of N keys, K and V) into a 2-3 stage ring.
@@ -56,8 +55,11 @@ namespace qkv {
 namespace {
 
 constexpr int kBM = 128;                     // query rows per CTA (MMA M)
-constexpr int kThreads = 512;                 // four warpgroups
-constexpr int kRegProducer = 96, kRegSoftmax = 160;   // 2 * 96 + 2 * 160 = 512 = 4 * 128 at launch
+constexpr int kThreads = 640;                 // five warpgroups
+constexpr int kKThreads = 224;                // K producers: warps 1-3 and warpgroup 4
+// Registers per thread after setmaxnreg: 2 * 128 * 144 + 3 * 128 * 64 = 61440 = 640 * 96, the
+// block's allocation at launch.
+constexpr int kRegProducer = 64, kRegSoftmax = 144;
 constexpr int kStagesMax = 3;                // packed-tile ring (INT2: 3 stages, INT4: 2)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when the max grows by more
 constexpr uint32_t kTmemCols = 512;
@@ -161,28 +163,28 @@ __device__ __forceinline__ uint32_t sub128(uint32_t v) {
   x = __hsub2(x, __floats2bfloat162_rn(128.f, 128.f));
   return *reinterpret_cast<uint32_t*>(&x);
 }
-template <int BITS>
-__device__ __forceinline__ void unpack_codes32(const uint8_t* codes, uint32_t (&out)[16]) {
-  if constexpr (BITS == 2) {
-    const uint2 w2 = *reinterpret_cast<const uint2*>(codes);
+template <int BITS> struct CodeVecT { using type = uint2; };   // 32 codes: 8 bytes (INT2)
+template <> struct CodeVecT<4> { using type = uint4; };            // 16 bytes (INT4)
+
+// Arguments by value: taking the address of a register copy would move it to local memory.
+__device__ __forceinline__ void unpack_codes32(uint2 w2, uint32_t (&out)[16]) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {     // one word = 16 codes = one channel block, code k at bits 2k
-      const uint32_t w = h ? w2.y : w2.x;
+  for (int h = 0; h < 2; ++h) {       // one word = 16 codes = one channel block, code k at bits 2k
+    const uint32_t w = h ? w2.y : w2.x;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) out[h * 8 + k] = sub128(((w >> (2 * k)) & 0x00030003u) | kCodeMagic);
-    }
-  } else {
-    const uint4 w4 = *reinterpret_cast<const uint4*>(codes);
+    for (int k = 0; k < 8; ++k) out[h * 8 + k] = sub128(((w >> (2 * k)) & 0x00030003u) | kCodeMagic);
+  }
+}
+__device__ __forceinline__ void unpack_codes32(uint4 w4, uint32_t (&out)[16]) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {     // two words = 16 codes = one channel block, code k at bits 4k
-      const uint32_t a = h ? w4.z : w4.x, b = h ? w4.w : w4.y;
-      const uint32_t lo = __byte_perm(a, b, 0x5410);   // codes 0-3 | codes 8-11 << 16
-      const uint32_t hi = __byte_perm(a, b, 0x7632);   // codes 4-7 | codes 12-15 << 16
+  for (int h = 0; h < 2; ++h) {       // two words = 16 codes = one channel block, code k at bits 4k
+    const uint32_t a = h ? w4.z : w4.x, b = h ? w4.w : w4.y;
+    const uint32_t lo = __byte_perm(a, b, 0x5410);   // codes 0-3 | codes 8-11 << 16
+    const uint32_t hi = __byte_perm(a, b, 0x7632);   // codes 4-7 | codes 12-15 << 16
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        out[h * 8 + k] = sub128(((lo >> (4 * k)) & 0x000F000Fu) | kCodeMagic);
-        out[h * 8 + 4 + k] = sub128(((hi >> (4 * k)) & 0x000F000Fu) | kCodeMagic);
-      }
+    for (int k = 0; k < 4; ++k) {
+      out[h * 8 + k] = sub128(((lo >> (4 * k)) & 0x000F000Fu) | kCodeMagic);
+      out[h * 8 + 4 + k] = sub128(((hi >> (4 * k)) & 0x000F000Fu) | kCodeMagic);
     }
   }
 }
@@ -195,42 +197,37 @@ __device__ __forceinline__ void permute16(const uint32_t* in, uint32_t* out) {
 
 // Dequantises 32 channels: x_hat = zp + step * code (fp32 FMA on a float whose mantissa holds the
 // code, 1 + code * 2^-k, so no integer conversion is needed), rounded to bf16.
-template <int BITS>
-__device__ __forceinline__ void dequant32(const uint8_t* codes, float step, float zp,
-                                          uint32_t (&out)[16]) {
-  if constexpr (BITS == 2) {
-    const uint2 w2 = *reinterpret_cast<const uint2*>(codes);
-    const float s16 = step * 16.f, s4 = step * 4.f;
-    const float c16 = zp - s16, c4 = zp - s4;
+__device__ __forceinline__ void dequant32(uint2 w2, float step, float zp, uint32_t (&out)[16]) {
+  const float s16 = step * 16.f, s4 = step * 4.f;
+  const float c16 = zp - s16, c4 = zp - s4;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t w = h ? w2.y : w2.x;   // 16 codes, code k at bits 2k
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t w = h ? w2.y : w2.x;   // 16 codes, code k at bits 2k
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const int sh = 19 - 4 * p;          // low code of the pair -> bits 19-20, high -> 21-22
-        const uint32_t s = sh >= 0 ? (w << sh) : (w >> (-sh));
-        const float lo = __uint_as_float((s & (3u << 19)) | 0x3F800000u);   // 1 + c/16
-        const float hi = __uint_as_float((s & (3u << 21)) | 0x3F800000u);   // 1 + c/4
-        const float2 x = __ffma2_rn(make_float2(s16, s4), make_float2(lo, hi), make_float2(c16, c4));
-        out[h * 8 + p] = pack_bf16x2(x.x, x.y);
-      }
+    for (int p = 0; p < 8; ++p) {
+      const int sh = 19 - 4 * p;          // low code of the pair -> bits 19-20, high -> 21-22
+      const uint32_t s = sh >= 0 ? (w << sh) : (w >> (-sh));
+      const float lo = __uint_as_float((s & (3u << 19)) | 0x3F800000u);   // 1 + c/16
+      const float hi = __uint_as_float((s & (3u << 21)) | 0x3F800000u);   // 1 + c/4
+      const float2 x = __ffma2_rn(make_float2(s16, s4), make_float2(lo, hi), make_float2(c16, c4));
+      out[h * 8 + p] = pack_bf16x2(x.x, x.y);
     }
-  } else {
-    const uint4 w4 = *reinterpret_cast<const uint4*>(codes);
-    const float s256 = step * 256.f, s16 = step * 16.f;
-    const float c256 = zp - s256, c16 = zp - s16;
+  }
+}
+__device__ __forceinline__ void dequant32(uint4 w4, float step, float zp, uint32_t (&out)[16]) {
+  const float s256 = step * 256.f, s16 = step * 16.f;
+  const float c256 = zp - s256, c16 = zp - s16;
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const uint32_t w = h == 0 ? w4.x : h == 1 ? w4.y : h == 2 ? w4.z : w4.w;  // 8 codes at 4k
+  for (int h = 0; h < 4; ++h) {
+    const uint32_t w = h == 0 ? w4.x : h == 1 ? w4.y : h == 2 ? w4.z : w4.w;  // 8 codes at 4k
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const int sh = 15 - 8 * p;          // low code -> bits 15-18, high -> 19-22
-        const uint32_t s = sh >= 0 ? (w << sh) : (w >> (-sh));
-        const float lo = __uint_as_float((s & (0xFu << 15)) | 0x3F800000u);  // 1 + c/256
-        const float hi = __uint_as_float((s & (0xFu << 19)) | 0x3F800000u);  // 1 + c/16
-        const float2 x = __ffma2_rn(make_float2(s256, s16), make_float2(lo, hi), make_float2(c256, c16));
-        out[h * 4 + p] = pack_bf16x2(x.x, x.y);
-      }
+    for (int p = 0; p < 4; ++p) {
+      const int sh = 15 - 8 * p;          // low code -> bits 15-18, high -> 19-22
+      const uint32_t s = sh >= 0 ? (w << sh) : (w >> (-sh));
+      const float lo = __uint_as_float((s & (0xFu << 15)) | 0x3F800000u);  // 1 + c/256
+      const float hi = __uint_as_float((s & (0xFu << 19)) | 0x3F800000u);  // 1 + c/16
+      const float2 x = __ffma2_rn(make_float2(s256, s16), make_float2(lo, hi), make_float2(c256, c16));
+      out[h * 4 + p] = pack_bf16x2(x.x, x.y);
     }
   }
 }
@@ -274,7 +271,7 @@ __device__ __forceinline__ void load_meta(const uint8_t* meta, int idx, float& s
 template <int D, int N, int kIters, int NT, bool kPermute>
 __device__ __forceinline__ void copy_rows(const uint4* src, uint8_t* tile, int valid, int t) {
   constexpr int kItems = N * (D / 32);
-  constexpr int kBatch = 2;                  // items in flight per thread (register budget)
+  constexpr int kBatch = 1;                  // items in flight per thread (register budget)
 #pragma unroll 1
   for (int i0 = 0; i0 < kIters; i0 += kBatch) {
     uint4 a[kBatch][4];
@@ -377,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
   constexpr int NH = N / 2;                   // keys of a tile per softmax warpgroup
   constexpr int kItems = N * (D / 32);        // (key, 32-channel block) items of one tile
   constexpr int kItersV = kItems / 128;       // per V-producer thread (128 threads)
-  constexpr int kItersK = (kItems + 95) / 96; // per K-producer thread (96 threads)
+  constexpr int kItersK = (kItems + kKThreads - 1) / kKThreads;   // per K-producer thread
   static_assert(kItems % 128 == 0 && kItersV % 2 == 0, "tile items must split evenly over a warpgroup");
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // 1024-byte alignment (128B-swizzle atoms) by offsetting the shared array itself, so that the
@@ -420,12 +417,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     *abort_flag = 0;
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_KH_FULL || i == B_KH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1) cnt = 3;
+      if (i == B_KH_FULL || i == B_KH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1) cnt = 7;
       if (i == B_VH_FULL || i == B_VH_FULL + 1) cnt = 4;
       if (i == B_KC_EMPTY || i == B_KC_EMPTY + 1 || i == B_S_FREE || i == B_S_FREE + 1 ||
           i == B_P_FULL || i == B_P_FULL + 1 || i == B_Q_FULL)
         cnt = 8;                                   // both softmax warpgroups
-      if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = 7;   // K and V producer warps
+      if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = 11;  // K and V producer warps
       mbar_init(bar(i), cnt);
     }
     mbar_init_fence();
@@ -444,13 +441,16 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t tm_q = tmem + kColQ, tm_o = tmem + kColO, tm_p = tmem + kColP;
       const uint32_t tm_s = tmem + kColS;
-      const uint64_t kdesc[2] = {smem_desc_sw128(smem_u32(smem + L.kt), 16u, 1024u),
-                                 smem_desc_sw128(smem_u32(smem + L.kt + C::kTile), 16u, 1024u)};
-      const uint64_t vdesc[2] = {smem_desc_sw128(smem_u32(smem + L.vt), C::kDblk, 1024u),
-                                 smem_desc_sw128(smem_u32(smem + L.vt + C::kTile), C::kDblk, 1024u)};
+      // Descriptors of buffer 0; buffer 1 is the same descriptor with its start address (bits 0-13,
+      // 16-byte units) advanced by the buffer size. Arithmetic, not an array indexed by the
+      // buffer, which would live in local memory.
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + L.kt), 16u, 1024u);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + L.vt), C::kDblk, 1024u);
       const uint64_t adesc = smem_desc_noswz(smem_u32(ax), 128u, 256u);
-      const uint64_t bdesc[2] = {smem_desc_noswz(smem_u32(bx), 128u, 256u),
-                                 smem_desc_noswz(smem_u32(bx + C::kBx), 128u, 256u)};
+      const uint64_t bdesc0 = smem_desc_noswz(smem_u32(bx), 128u, 256u);
+      auto kdesc = [&](int b) { return kdesc0 + static_cast<uint64_t>(b) * (C::kTile >> 4); };
+      auto vdesc = [&](int b) { return vdesc0 + static_cast<uint64_t>(b) * (C::kTile >> 4); };
+      auto bdesc = [&](int b) { return bdesc0 + static_cast<uint64_t>(b) * (C::kBx >> 4); };
       // O += P_i V_i once the softmax wrote P_i and V_i is in smem.
       auto issue_pv = [&](int i) -> bool {
         const int vb = i & 1, pb = i % C::kPB;
@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk)   // 16 keys = two 1024-byte atoms per step
-          mma_ts(tm_o, tm_p + pb * (N / 2) + kk * 8u, vdesc[vb] + kk * (2048u >> 4), idesc_pv,
+          mma_ts(tm_o, tm_p + pb * (N / 2) + kk * 8u, vdesc(vb) + kk * (2048u >> 4), idesc_pv,
                  (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(bar(B_VH_EMPTY + vb));
         tc_commit(bar(B_PV_DONE + pb));
@@ -484,13 +484,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
 #pragma unroll
           for (int g = 0; g < NG; ++g) {
             const int ch = g * C::G + kk * 16;
-            mma_ts(tm_sj + g * N, tm_q + ch / 2, kdesc[kb] + kofs(ch), idesc_s, kk > 0 ? 1u : 0u);
+            mma_ts(tm_sj + g * N, tm_q + ch / 2, kdesc(kb) + kofs(ch), idesc_s, kk > 0 ? 1u : 0u);
           }
         if (j < Tc) {
           // zero-point and correction terms: row extras x key extras (no swizzle, K-major)
 #pragma unroll
           for (int g = 0; g < NG; ++g)
-            mma_ss(tm_sj + g * N, adesc + g * ((kBM * 32) >> 4), bdesc[kb] + g * ((N * 32) >> 4), idesc_s, 1u);
+            mma_ss(tm_sj + g * N, adesc + g * ((kBM * 32) >> 4), bdesc(kb) + g * ((N * 32) >> 4), idesc_s, 1u);
         }
         tc_commit(bar(B_KH_EMPTY + kb));
         tc_commit(bar(B_S_FULL + sb));
@@ -502,10 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       mbar_wait_drain(bar(B_DRAIN), 0);
     }
     __syncwarp();
-  } else if (wg == 0) {
+  } else if (wg == 0 || wg == 4) {
     // ---------------------------------------------------------------- K operand tiles (warps 1-3)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
-    const int t = threadIdx.x - 32;
+    const int t = wg == 0 ? threadIdx.x - 32 : threadIdx.x - 512 + 96;   // 0 .. kKThreads - 1
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* kt = smem + L.kt + sb * C::kTile;
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const int valid = static_cast<int>(rem < N ? rem : N);
         const uint8_t* kcodes = smem + L.pk + s * L.stage;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
-        using CodeVec = typename std::conditional<BITS == 2, uint2, uint4>::type;
+        using CodeVec = typename CodeVecT<BITS>::type;
         // Two items per iteration, the loop itself not unrolled: the code of all four roles has
         // to share the instruction caches of each SM sub-partition.
 #pragma unroll 1
@@ -524,17 +524,17 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           CodeVec cv[2];
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            const int it = t + 96 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
-            if (it < kItems)
+            const int it = t + kKThreads * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+            if (i0 + i < kItersK && it < kItems)
               cv[i] = *reinterpret_cast<const CodeVec*>(kcodes + key * (D * BITS / 8) + blk * (4 * BITS));
           }
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            const int it = t + 96 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
-            if (it >= kItems) break;
+            const int it = t + kKThreads * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
+            if (i0 + i >= kItersK || it >= kItems) break;
             uint32_t v[16];
             if (key < valid) {
-              unpack_codes32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), v);
+              unpack_codes32(cv[i], v);
             } else {
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0u;
@@ -547,10 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
         const uint8_t* kmeta = kcodes + C::kCodes;
         float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
-        constexpr int kItersC = (N * NG + 95) / 96;
+        constexpr int kItersC = (N * NG + kKThreads - 1) / kKThreads;
 #pragma unroll
         for (int i = 0; i < kItersC; ++i) {
-          const int e = t + 96 * i;
+          const int e = t + kKThreads * i;
           if (e >= N * NG) break;
           const int key = e / NG, g = e % NG;
           float a = 0.f, rho = 0.f, sigma = 0.f;
@@ -583,14 +583,14 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
         const uint4* src = reinterpret_cast<const uint4*>(p.K_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
-        copy_rows<D, N, kItersK, 96, true>(src, kt, valid, t);
+        copy_rows<D, N, kItersK, kKThreads, true>(src, kt, valid, t);
         fence_async_smem();
         // Scales of the current tile: the plain score scale for every key and group, so that the
         // softmax forms every tile's scores the same way.
         if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
         float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
 #pragma unroll 1
-        for (int e = t; e < static_cast<int>(C::kKconst / 4); e += 96) kc[e] = p.scale_log2;
+        for (int e = t; e < static_cast<int>(C::kKconst / 4); e += kKThreads) kc[e] = p.scale_log2;
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(bar(B_KH_FULL + sb));
@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const uint8_t* vcodes = smem + L.pk + s * L.stage + C::kCodes + L.meta;
         const uint8_t* vmeta = vcodes + C::kCodes;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
-        using CodeVec = typename std::conditional<BITS == 2, uint2, uint4>::type;
+        using CodeVec = typename CodeVecT<BITS>::type;
         constexpr int kBatch = 2;                 // items per iteration; the loop is not unrolled
 #pragma unroll 1
         for (int i0 = 0; i0 < kItersV; i0 += kBatch) {
@@ -655,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
             const int it = t + 128 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
             uint32_t v[16];
             if (key < valid) {
-              dequant32<BITS>(reinterpret_cast<const uint8_t*>(&cv[i]), st[i], zp[i], v);
+              dequant32(cv[i], st[i], zp[i], v);
             } else {
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0u;
