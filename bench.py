@@ -224,6 +224,50 @@ def oracle_sample(w, x_cpu, budget_s: float, seed: int = 0):
 
 
 # ------------------------------------------------------------------------------------ GPU arm
+def decode_sweep(dev, peaks, flush, steps: int = 20):
+    """Few query rows per KV head over the chunked-prefill workload's 131072-token INT2 cache
+    (B4, 32 query / 8 KV heads): the regime where attention reads the packed cache once and the
+    cached keys are split over CTAs. Packed-cache GB/s against the measured HBM peak."""
+    base = WORKLOADS["prefill_gqa"]
+    x = make_inputs(base.with_(Lq=16, Lcur=16), device=dev)
+    cache = api.KVCache(base.B, base.Hkv, base.d, base.bits, base.group, api.round_capacity(base.Lc),
+                        base.meta, device=dev)
+    for t0 in range(0, base.Lc, 16384):
+        api.kv_quantize_append(cache, x["K_src"][:, :, t0:t0 + 16384].contiguous(),
+                               x["V_src"][:, :, t0:t0 + 16384].contiguous())
+    stream = torch.cuda.current_stream(dev)
+    out = {"workload": "prefill_gqa cache (B4 Hq32 Hkv8 d128 Lc131072 INT2 G64 f32 meta), Lcur = Lq, causal",
+           "bound": "hbm", "peak_gbs": float(peaks["hbm_gbs"]), "points": []}
+    for Lq in (1, 4, 16):
+        Q = x["Q"][:, :, :Lq].contiguous()
+        Kc = x["K_cur"][:, :, :Lq].contiguous()
+        Vc = x["V_cur"][:, :, :Lq].contiguous()
+        O = torch.empty_like(Q)
+        L = torch.empty(base.B, base.Hq, Lq, dtype=torch.float32, device=dev)
+        nws = api.attention_workspace_bytes(cache, base.Hq, Lq, Lq)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+        ts = []
+        for i in range(steps + 3):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            api.corrected_attention(Q, cache, Kc, Vc, correct=1, causal=True, out=O, lse=L, workspace=ws)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        gbs = cache.packed_bytes(base.Lc) / (ms * 1e-3) / 1e9
+        out["points"].append({"Lq": Lq, "rows_per_kv_head": 4 * Lq, "ms": round(ms, 4),
+                              "workspace_bytes": nws, "packed_cache_gbs": round(gbs, 1),
+                              "frac": round(gbs / float(peaks["hbm_gbs"]), 4)})
+    if api.device_status() != 0:
+        raise RuntimeError("device status after the decode sweep")
+    del x, cache
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     w = WORKLOADS[args.workload]
     torch.cuda.set_device(local)
@@ -366,6 +410,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 2 * K,
         "clocks": clocks.summary(),
     }
+    if not args.no_decode:
+        result["decode"] = decode_sweep(dev, peaks, flush)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         x_cpu = make_inputs(w, device="cpu")
         est_s, full_flops, text, cores = oracle_sample(w, x_cpu, args.cpu_budget)
@@ -407,6 +453,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the few-query-rows (decode) sweep")
     ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
                     help="store the DRAM bytes per launch of an ncu report (taken on --workload) and exit")
     ap.add_argument("--record-command", default="", help="the command line that made the report")

@@ -93,7 +93,13 @@ qkv_status qkv_cache_bytes(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int
 qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const void* V, int32_t in_dtype,
                               int64_t L_new, void* stream);
 
-/* Device workspace that corrected_attention needs for this shape (may be 0). */
+/*
+ * Device workspace with which corrected_attention splits the cached keys of each (batch, KV head)
+ * over several CTAs (0 when the shape fills the GPU without a split). A split is chosen when the
+ * query rows of a KV head fill few 128-row tiles (few query rows per KV head, e.g. decoding), so
+ * that more SMs share the cache reads; its partial results, n_split * B * H_q * L_q * (d + 1) fp32
+ * values, are then merged by a second kernel. The size depends on the GPU's SM count.
+ */
 qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H_q, int64_t L_q,
                                                int64_t L_cur, size_t* bytes);
 
@@ -112,8 +118,9 @@ qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H
  *  scale        : score scale; <= 0 means 1/sqrt(d).
  *  O            : dtype [B][H_q][L_q][d] (same type as Q). LSE: fp32 [B][H_q][L_q], natural log
  *                 of the row's softmax denominator (-inf and O = 0 for a row that sees no key).
- *  workspace    : device scratch of at least corrected_attention_workspace_bytes() (may be NULL
- *                 when that is 0).
+ *  workspace    : device scratch of corrected_attention_workspace_bytes() bytes, 16-byte aligned,
+ *                 owned by the caller; NULL (or too small) runs the same attention without the
+ *                 key split. Calls on one stream may reuse it; concurrent calls need their own.
  * L_cur = 0 and cache->length = 0 together are rejected (no keys at all).
  */
 qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,

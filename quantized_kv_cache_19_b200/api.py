@@ -173,8 +173,13 @@ def kv_quantize_append(cache: KVCache, K: torch.Tensor, V: torch.Tensor) -> None
 def corrected_attention(Q: torch.Tensor, cache: KVCache, K_cur: Optional[torch.Tensor],
                         V_cur: Optional[torch.Tensor], correct: int = 1, causal: bool = False,
                         scale: float = 0.0, out: Optional[torch.Tensor] = None,
-                        lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """O [B][H_q][L_q][d] (Q's dtype) and LSE [B][H_q][L_q] (fp32) of the corrected attention."""
+                        lse: Optional[torch.Tensor] = None,
+                        workspace="auto") -> Tuple[torch.Tensor, torch.Tensor]:
+    """O [B][H_q][L_q][d] (Q's dtype) and LSE [B][H_q][L_q] (fp32) of the corrected attention.
+
+    workspace: "auto" allocates the scratch the library asks for (a key split for shapes with few
+    query rows per KV head); None runs without it (no split); a uint8 CUDA tensor is used as is.
+    """
     _need_cuda(Q, K_cur, V_cur, out, lse)
     B, Hq, Lq, d = Q.shape
     Lcur = 0 if K_cur is None else K_cur.shape[2]
@@ -187,12 +192,26 @@ def corrected_attention(Q: torch.Tensor, cache: KVCache, K_cur: Optional[torch.T
     lib = load_library()
     ws = ctypes.c_size_t()
     _check(lib.corrected_attention_workspace_bytes(ctypes.byref(cache.desc), Hq, Lq, Lcur, ctypes.byref(ws)))
-    work = torch.empty(ws.value, dtype=torch.uint8, device=Q.device) if ws.value else None
+    if isinstance(workspace, torch.Tensor):
+        _need_cuda(workspace)
+        work, nbytes = workspace, workspace.numel() * workspace.element_size()
+    elif workspace == "auto" and ws.value:
+        work, nbytes = torch.empty(ws.value, dtype=torch.uint8, device=Q.device), ws.value
+    else:
+        work, nbytes = None, 0
     _check(lib.corrected_attention(_ptr(Q), _DTYPE[Q.dtype], Hq, Lq, ctypes.byref(cache.desc),
                                    _ptr(K_cur), _ptr(V_cur), Lcur, int(correct), int(bool(causal)),
-                                   float(scale), _ptr(out), _ptr(lse), _ptr(work), ws.value,
+                                   float(scale), _ptr(out), _ptr(lse), _ptr(work), nbytes,
                                    _stream(Q.device)))
     return out, lse
+
+
+def attention_workspace_bytes(cache: KVCache, Hq: int, Lq: int, Lcur: int) -> int:
+    """Scratch bytes with which corrected_attention splits the cached keys (0: no split)."""
+    lib = load_library()
+    ws = ctypes.c_size_t()
+    _check(lib.corrected_attention_workspace_bytes(ctypes.byref(cache.desc), Hq, Lq, Lcur, ctypes.byref(ws)))
+    return int(ws.value)
 
 
 def jensen_bias(Q: torch.Tensor, cache: KVCache, scale: float = 0.0) -> torch.Tensor:

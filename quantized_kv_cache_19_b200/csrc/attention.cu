@@ -401,7 +401,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
   const int64_t rows_total = static_cast<int64_t>(p.r) * p.Lq;
 
   // Tiles: cached ones first, then current ones (causal: only those some row of this CTA sees).
-  const int Tc = static_cast<int>((p.Lc + N - 1) / N);
+  // With a split over the cached keys, this CTA takes cached tiles [c0, c0 + Tc) and, if it is the
+  // last split, the current chunk.
+  const int Tc_all = static_cast<int>((p.Lc + N - 1) / N);
+  const int split = blockIdx.z;
+  const int c0 = static_cast<int>(static_cast<int64_t>(split) * Tc_all / gridDim.z);
+  const int Tc = static_cast<int>(static_cast<int64_t>(split + 1) * Tc_all / gridDim.z) - c0;
+  const bool last_split = split == static_cast<int>(gridDim.z) - 1;
   int64_t cur_keys = p.Lcur;
   if (p.causal) {
     const int64_t R0 = static_cast<int64_t>(m_tile) * kBM;
@@ -410,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     const int64_t lim = max_i + 1 + (p.Lcur - p.Lq);
     cur_keys = lim < 0 ? 0 : (lim < p.Lcur ? lim : p.Lcur);
   }
-  const int Tn = static_cast<int>((cur_keys + N - 1) / N);
+  const int Tn = last_split ? static_cast<int>((cur_keys + N - 1) / N) : 0;
   const int T = Tc + Tn;
 
   if (threadIdx.x == 0) {
@@ -512,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       if (!warp_wait(bar(B_KH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
       if (j < Tc) {
         const int s = j % kStages, k = j / kStages;
-        const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
+        const int64_t rem = p.Lc - static_cast<int64_t>(c0 + j) * N;
         const int valid = static_cast<int>(rem < N ? rem : N);
         const uint8_t* kcodes = smem + L.pk + s * L.stage;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
@@ -611,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       const int s = next_load % kStages, k = next_load / kStages;
       if (!mbar_wait(bar(B_PK_EMPTY + s), (k & 1) ^ 1, abort_flag, p.status)) return false;
       const uint32_t dst = smem_u32(smem + L.pk + s * L.stage);
-      const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(next_load) * N;
+      const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(c0 + next_load) * N;
       const uint32_t fb = bar(B_PK_FULL + s);
       mbar_arrive_expect_tx(fb, 2 * (C::kCodes + L.meta));
       bulk_g2s(dst, p.k_codes + row0 * row_codes, C::kCodes, fb);
@@ -631,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       if (!warp_wait(bar(B_VH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
       if (j < Tc) {
         const int s = j % kStages, k = j / kStages;
-        const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
+        const int64_t rem = p.Lc - static_cast<int64_t>(c0 + j) * N;
         const int valid = static_cast<int>(rem < N ? rem : N);
         const uint8_t* vcodes = smem + L.pk + s * L.stage + C::kCodes + L.meta;
         const uint8_t* vmeta = vcodes + C::kCodes;
@@ -774,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       float2 s2[NH / 2];         // scores of this half's key pairs (log2 units)
       int valid;                 // keys of the whole tile that count for this row
       if (cached) {
-        const int64_t rem = p.Lc - static_cast<int64_t>(j) * N;
+        const int64_t rem = p.Lc - static_cast<int64_t>(c0 + j) * N;
         valid = static_cast<int>(rem < N ? rem : N);
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
@@ -901,6 +907,8 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     const float l_tot = l_run + xsum[(half ^ 1) * kBM + row];
     const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
     uint8_t* orow = static_cast<uint8_t*>(p.O) + out_row * D * 2 + half * D;
+    const bool partial = gridDim.z > 1;
+    float* prow = partial ? p.ws_o + (static_cast<int64_t>(split) * p.rows_all + out_row) * D + half * (D / 2) : nullptr;
 #pragma unroll
     for (int c = 0; c < D / 2; c += 32) {
       uint32_t r[32];
@@ -911,7 +919,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
 #pragma unroll
         for (int k = 0; k < 32; ++k) r[k] = 0u;
       }
-      if (valid_row) {
+      if (valid_row && partial) {
+        float4* dst = reinterpret_cast<float4*>(prow + c);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dst[k] = make_float4(__uint_as_float(r[4 * k]) * inv_l, __uint_as_float(r[4 * k + 1]) * inv_l,
+                               __uint_as_float(r[4 * k + 2]) * inv_l, __uint_as_float(r[4 * k + 3]) * inv_l);
+      } else if (valid_row) {
         uint4* dst = reinterpret_cast<uint4*>(orow) + c / 8;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -926,7 +940,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     }
     if (valid_row && half == 0) {
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      p.LSE[out_row] = l_tot > 0.f ? (m_use + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+      const float lse = l_tot > 0.f ? (m_use + __log2f(l_tot)) * 0.69314718055994530942f : -INFINITY;
+      if (partial) p.ws_lse[static_cast<int64_t>(split) * p.rows_all + out_row] = lse;
+      else p.LSE[out_row] = lse;
     }
   }
 
@@ -949,7 +965,8 @@ cudaError_t launch_impl(const AttnParams& p, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(p.r) * p.Lq;
-  dim3 grid(static_cast<unsigned>((rows + kBM - 1) / kBM), static_cast<unsigned>(p.B * p.Hkv));
+  dim3 grid(static_cast<unsigned>((rows + kBM - 1) / kBM), static_cast<unsigned>(p.B * p.Hkv),
+            static_cast<unsigned>(p.n_split > 1 ? p.n_split : 1));
   corrected_attention_kernel<D, BITS, NG><<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
@@ -965,6 +982,8 @@ cudaError_t launch_groups(const AttnParams& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int attention_tile_keys(int n_groups) { return n_groups == 4 ? 64 : 128; }
 
 cudaError_t launch_attention_bf16(const AttnParams& p, int d, int bits, cudaStream_t stream) {
   if (d == 128) return bits == 2 ? launch_groups<128, 2>(p, stream) : launch_groups<128, 4>(p, stream);

@@ -149,6 +149,34 @@ QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const voi
   return QKV_OK;
 }
 
+// Splits of the cached keys for the bf16 kernel: used only when the (row tile, batch * KV head)
+// grid would leave more than half of the SMs idle (few query rows per KV head, e.g. decoding);
+// each split then keeps at least one key tile. 1 = no split.
+static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
+  if (L_q <= 0 || c->length <= 0) return 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  const int64_t rows = static_cast<int64_t>(H_q / c->H_kv) * L_q;
+  const int64_t ctas = (rows + 127) / 128 * c->B * c->H_kv;
+  const int tile = attention_tile_keys(c->d / c->group);
+  const int64_t tiles = (c->length + tile - 1) / tile;
+  if (ctas * 2 > sms || tiles < 2) return 1;
+  int64_t n = sms / ctas;
+  if (n > tiles) n = tiles;
+  if (n > 32) n = 32;
+  return n < 1 ? 1 : static_cast<int>(n);
+}
+
+static size_t split_workspace_bytes(const qkv_cache* c, int32_t H_q, int64_t L_q, int n) {
+  if (n <= 1) return 0;
+  const size_t rows_all = static_cast<size_t>(c->B) * H_q * L_q;
+  return static_cast<size_t>(n) * rows_all * (static_cast<size_t>(c->d) + 1) * sizeof(float);
+}
+
 QKV_API qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H_q,
                                                        int64_t L_q, int64_t L_cur, size_t* bytes) {
   t_last_error.clear();
@@ -157,7 +185,7 @@ QKV_API qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, i
   if (!bytes) return fail(QKV_ERR_INVALID_ARG, "NULL output");
   if (H_q < 1 || H_q % cache->H_kv || L_q < 0 || L_cur < 0)
     return fail(QKV_ERR_INVALID_ARG, "bad H_q / L_q / L_cur");
-  *bytes = 0;
+  *bytes = split_workspace_bytes(cache, H_q, L_q, attention_splits(cache, H_q, L_q));
   return QKV_OK;
 }
 
@@ -167,8 +195,6 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
                                        int32_t causal_cur, float scale, void* O, float* LSE,
                                        void* workspace, size_t workspace_bytes, void* stream) {
   t_last_error.clear();
-  (void)workspace;
-  (void)workspace_bytes;
   qkv_status s = check_cache(cache);
   if (s != QKV_OK) return s;
   if (!in_dtype_ok(dtype)) return fail(QKV_ERR_UNSUPPORTED, "dtype must be F32 or BF16");
@@ -206,9 +232,31 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   p.scale_log2 = sc * log2e;
   p.wcoef_log2 = sc * sc / 24.0f * log2e;
   p.inv_scale_log2 = 1.0f / (sc * log2e);
-  e = dtype == QKV_F32 ? launch_attention_f32(p, cache->d, cache->bits, static_cast<cudaStream_t>(stream))
-                       : launch_attention_bf16(p, cache->d, cache->bits, static_cast<cudaStream_t>(stream));
+  p.n_split = 1;
+  p.rows_all = static_cast<int64_t>(cache->B) * H_q * L_q;
+  p.ws_o = nullptr;
+  p.ws_lse = nullptr;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == QKV_F32) {
+    e = launch_attention_f32(p, cache->d, cache->bits, st);
+    if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");
+    return QKV_OK;
+  }
+  // Split over the cached keys when the caller gave the workspace for it; without it the same
+  // result comes from the unsplit kernel.
+  const int n = attention_splits(cache, H_q, L_q);
+  const size_t need = split_workspace_bytes(cache, H_q, L_q, n);
+  if (n > 1 && workspace && workspace_bytes >= need && aligned16(workspace)) {
+    p.n_split = n;
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_lse = p.ws_o + static_cast<size_t>(n) * p.rows_all * cache->d;
+  }
+  e = launch_attention_bf16(p, cache->d, cache->bits, st);
   if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");
+  if (p.n_split > 1) {
+    e = launch_split_merge(p.ws_o, p.ws_lse, p.n_split, p.rows_all, cache->d, O, LSE, st);
+    if (e != cudaSuccess) return cuda_fail(e, "corrected_attention merge launch");
+  }
   return QKV_OK;
 }
 

@@ -46,9 +46,21 @@ struct AttnParams {
   float scale_log2;   // score scale * log2(e)
   float wcoef_log2;   // scale^2 / 24 * log2(e): Jensen-correction coefficient in log2 units
   float inv_scale_log2;  // 1 / (scale * log2(e))
+  // Split over the cached keys (n_split > 1): CTA z takes cached tiles [z * T / n, (z+1) * T / n)
+  // (the last one also the current chunk) and writes its row's normalised partial output and
+  // log-sum-exp to ws_o [n_split][rows_all][d] and ws_lse [n_split][rows_all] (fp32).
+  int n_split;
+  int64_t rows_all;     // B * Hq * Lq
+  float* ws_o;
+  float* ws_lse;
 };
 // bf16 inputs: tcgen05 kernel. fp32 inputs: CUDA-core fp32 kernel.
 cudaError_t launch_attention_bf16(const AttnParams& p, int d, int bits, cudaStream_t stream);
+// Key tiles of one (batch, KV head) in the bf16 kernel (128 keys, or 64 with four groups).
+int attention_tile_keys(int n_groups);
+// Merge of split partials: O (bf16) and LSE from ws_o / ws_lse.
+cudaError_t launch_split_merge(const float* ws_o, const float* ws_lse, int n_split, int64_t rows_all,
+                               int d, void* O, float* LSE, cudaStream_t stream);
 cudaError_t launch_attention_f32(const AttnParams& p, int d, int bits, cudaStream_t stream);
 
 // Jensen-correction term alone: bias[B][Hq][Lq][Lc] (natural units).
