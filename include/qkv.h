@@ -130,6 +130,26 @@ qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_
                                void* stream);
 
 /*
+ * corrected_attention for callers that cannot allocate device memory. (The pages have no
+ * counterpart: this is an interface of this library.) Same arguments and results as
+ * corrected_attention, without the workspace: when the shape splits its cached keys, the partial
+ * results go to a scratch array that the library itself holds in device memory, 8 MiB on every GPU
+ * that loads the library, kept until the process exits. No call allocates or frees memory.
+ *  - A shape whose split needs more than 8 MiB of scratch (corrected_attention_workspace_bytes()
+ *    larger than 8 MiB) is rejected with QKV_ERR_UNSUPPORTED; corrected_attention with a workspace
+ *    handles it.
+ *  - The first call on a device that needs the scratch looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array: every value a call reads from it was written by the same call,
+ *    but two calls that overlap on the GPU (different streams, or different host threads) race on
+ *    it and must be serialised by the caller.
+ */
+qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                                       const qkv_cache* cache, const void* K_cur, const void* V_cur,
+                                       int64_t L_cur, int32_t correct, int32_t causal_cur, float scale,
+                                       void* O, float* LSE, void* stream);
+
+/*
  * The correction term alone, for checking: bias fp32 [B][H_q][L_q][cache->length] with
  * bias[b][hq][i][j] = (scale^2/24) * sum_c Q[b][hq][i][c]^2 * step_{j, c/group}^2, computed by
  * the same device functions corrected_attention uses (fp32).

@@ -58,6 +58,10 @@ _SIGS = {
                                            ctypes.POINTER(QkvCacheDesc), _P, _P, ctypes.c_int64,
                                            ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P,
                                            ctypes.c_size_t, _P]),
+    "corrected_attention_noalloc": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
+                                                   ctypes.POINTER(QkvCacheDesc), _P, _P, ctypes.c_int64,
+                                                   ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P,
+                                                   _P]),
     "qkv_jensen_bias": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
                                        ctypes.POINTER(QkvCacheDesc), ctypes.c_float, _P, _P]),
     "qkv_device_status": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
@@ -203,6 +207,31 @@ def corrected_attention(Q: torch.Tensor, cache: KVCache, K_cur: Optional[torch.T
                                    _ptr(K_cur), _ptr(V_cur), Lcur, int(correct), int(bool(causal)),
                                    float(scale), _ptr(out), _ptr(lse), _ptr(work), nbytes,
                                    _stream(Q.device)))
+    return out, lse
+
+
+def corrected_attention_noalloc(Q: torch.Tensor, cache: KVCache, K_cur: Optional[torch.Tensor],
+                                V_cur: Optional[torch.Tensor], correct: int = 1, causal: bool = False,
+                                scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """corrected_attention through the entry point that allocates nothing (library-owned scratch).
+
+    For callers that may not allocate device memory; only O and LSE are allocated here when not
+    given. Calls that overlap on the GPU share the library's scratch and must not run concurrently.
+    """
+    _need_cuda(Q, K_cur, V_cur, out, lse)
+    B, Hq, Lq, d = Q.shape
+    Lcur = 0 if K_cur is None else K_cur.shape[2]
+    if K_cur is not None and (K_cur.dtype != Q.dtype or V_cur.dtype != Q.dtype):
+        raise ValueError("K_cur, V_cur must have Q's dtype")
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=Q.device)
+    lib = load_library()
+    _check(lib.corrected_attention_noalloc(_ptr(Q), _DTYPE[Q.dtype], Hq, Lq, ctypes.byref(cache.desc),
+                                           _ptr(K_cur), _ptr(V_cur), Lcur, int(correct), int(bool(causal)),
+                                           float(scale), _ptr(out), _ptr(lse), _stream(Q.device)))
     return out, lse
 
 

@@ -306,3 +306,108 @@ QKV_API qkv_status qkv_device_status(int32_t reset, int32_t* code) {
   *code = v;
   return QKV_OK;
 }
+
+// ------------------------------------------------------------------ allocation-free attention
+// Some callers cannot allocate device memory at all: a host runtime whose device memory belongs to
+// another allocator and forbids allocations outside it, or a service that must not allocate once
+// it has started. For them corrected_attention_noalloc takes its key-split scratch from one
+// fixed-size array that the library itself owns in device memory (a file-scope __device__ array,
+// reserved on every GPU that loads the library until the process exits), so the call needs no
+// workspace argument and allocates nothing.
+//
+// In host code the array's name is only a host-side stand-in, not a device address: a kernel given
+// it would fault or, where the GPU can reach host memory, silently use the wrong memory. Its device
+// address is therefore looked up with cudaGetSymbolAddress, once per device with that device
+// current (on the entry point's first call on the device that needs the scratch), and passed to
+// the kernels.
+static constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+static float* noalloc_scratch(cudaError_t* err) {
+  static float* addr[64] = {nullptr};
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= 64) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<float*>(p);
+  }
+  return addr[dev];
+}
+
+QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                                               const qkv_cache* cache, const void* K_cur,
+                                               const void* V_cur, int64_t L_cur, int32_t correct,
+                                               int32_t causal_cur, float scale, void* O, float* LSE,
+                                               void* stream) {
+  t_last_error.clear();
+  qkv_status s = check_cache(cache);
+  if (s != QKV_OK) return s;
+  if (!in_dtype_ok(dtype)) return fail(QKV_ERR_UNSUPPORTED, "dtype must be F32 or BF16");
+  if (H_q < 1 || H_q % cache->H_kv)
+    return fail(QKV_ERR_INVALID_ARG, "H_q %d must be a positive multiple of H_kv %d", H_q,
+                cache->H_kv);
+  if (L_q < 0 || L_cur < 0) return fail(QKV_ERR_INVALID_ARG, "negative length");
+  if (correct != 0 && correct != 1) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0 or 1");
+  if (causal_cur != 0 && causal_cur != 1) return fail(QKV_ERR_INVALID_ARG, "causal_cur must be 0 or 1");
+  if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
+  if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
+  if (L_q == 0) return QKV_OK;
+  if (!Q || !O || !LSE) return fail(QKV_ERR_INVALID_ARG, "Q, O or LSE is NULL");
+  if (L_cur > 0 && (!K_cur || !V_cur)) return fail(QKV_ERR_INVALID_ARG, "K_cur or V_cur is NULL");
+  if (!aligned16(Q) || !aligned16(O) || !aligned16(LSE) || (L_cur > 0 && (!aligned16(K_cur) || !aligned16(V_cur))))
+    return fail(QKV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(H_q / cache->H_kv) * L_q;
+  if ((rows + 127) / 128 > 2147483647LL || static_cast<int64_t>(cache->B) * cache->H_kv > 65535)
+    return fail(QKV_ERR_UNSUPPORTED, "grid too large");
+  // The key split this shape takes, and whether its scratch fits the library's array.
+  const int n = dtype == QKV_BF16 ? attention_splits(cache, H_q, L_q) : 1;
+  const size_t need = split_workspace_bytes(cache, H_q, L_q, n);
+  if (need > kNoAllocScratchBytes)
+    return fail(QKV_ERR_UNSUPPORTED,
+                "this shape splits its cached keys %d ways and needs %zu bytes of scratch; the "
+                "library's static scratch holds %zu bytes (use corrected_attention with a workspace)",
+                n, need, kNoAllocScratchBytes);
+  cudaError_t e;
+  int* status = status_word(&e);
+  if (!status) return cuda_fail(e, "device status word");
+  float* scratch = nullptr;
+  if (n > 1) {
+    scratch = noalloc_scratch(&e);
+    if (!scratch) return cuda_fail(e, "address of the static scratch");
+  }
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(cache->d));
+  const float log2e = 1.4426950408889634f;
+  AttnParams p;
+  p.Q = Q; p.K_cur = K_cur; p.V_cur = V_cur; p.O = O; p.LSE = LSE;
+  p.k_codes = cache->k_codes; p.v_codes = cache->v_codes;
+  p.k_meta = cache->k_meta; p.v_meta = cache->v_meta;
+  p.status = status;
+  p.Lq = L_q; p.Lc = cache->length; p.Lcur = L_cur; p.capacity = cache->capacity;
+  p.B = cache->B; p.Hq = H_q; p.Hkv = cache->H_kv; p.r = H_q / cache->H_kv;
+  p.group = cache->group; p.n_groups = cache->d / cache->group;
+  p.correct = correct; p.causal = causal_cur;
+  p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
+  p.scale_log2 = sc * log2e;
+  p.wcoef_log2 = sc * sc / 24.0f * log2e;
+  p.inv_scale_log2 = 1.0f / (sc * log2e);
+  p.n_split = n;
+  p.rows_all = static_cast<int64_t>(cache->B) * H_q * L_q;
+  p.ws_o = scratch;
+  p.ws_lse = scratch ? scratch + static_cast<size_t>(n) * p.rows_all * cache->d : nullptr;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  e = dtype == QKV_F32 ? launch_attention_f32(p, cache->d, cache->bits, st)
+                       : launch_attention_bf16(p, cache->d, cache->bits, st);
+  if (e != cudaSuccess) return cuda_fail(e, "corrected_attention_noalloc launch");
+  if (n > 1) {
+    e = launch_split_merge(p.ws_o, p.ws_lse, n, p.rows_all, cache->d, O, LSE, st);
+    if (e != cudaSuccess) return cuda_fail(e, "corrected_attention_noalloc merge launch");
+  }
+  return QKV_OK;
+}
