@@ -400,6 +400,7 @@ def run_ours(args, world, rank, local):
                          "frac": round(qa_bytes / (mean_qa * 1e-3) / 1e9 / float(peaks["hbm_gbs"]), 4),
                          "full_cache": {"tokens": w.Lc, "ms_per_launch": round(full_ms, 5),
                                         "bytes_per_launch": full_bytes,
+                                        "traffic": ncu_traffic("quantize_append_kernel", w.name + "/full_cache"),
                                         "achieved_gbs": round(full_bytes / (full_ms * 1e-3) / 1e9, 1),
                                         "frac": round(full_bytes / (full_ms * 1e-3) / 1e9 /
                                                       float(peaks["hbm_gbs"]), 4)}},
@@ -457,9 +458,10 @@ def main(argv=None):
     ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
                     help="store the DRAM bytes per launch of an ncu report (taken on --workload) and exit")
     ap.add_argument("--record-command", default="", help="the command line that made the report")
+    ap.add_argument("--record-key", default=None, help="key to store the figures under (default: --workload)")
     args = ap.parse_args(argv)
     if args.record_traffic:
-        record_traffic(args.record_traffic, args.workload, args.record_command)
+        record_traffic(args.record_traffic, args.record_key or args.workload, args.record_command)
         return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
