@@ -523,30 +523,30 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const uint8_t* kcodes = smem + L.pk + s * L.stage;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
         using CodeVec = typename CodeVecT<BITS>::type;
-        // Two items per iteration, the loop itself not unrolled: the code of all four roles has
-        // to share the instruction caches of each SM sub-partition.
+        // One item per iteration with the next item's codes already loaded (shared-memory loads
+        // take ~170 cycles while the tensor core reads its operands), the loop itself not
+        // unrolled: the code of all roles shares the instruction caches of each SM sub-partition.
+        auto load_codes = [&](int it) {
+          return *reinterpret_cast<const CodeVec*>(kcodes + item_key<D>(it) * (D * BITS / 8) +
+                                                   item_blk<D>(it) * (4 * BITS));
+        };
+        CodeVec cv_next = load_codes(t < kItems ? t : 0);
 #pragma unroll 1
-        for (int i0 = 0; i0 < kItersK; i0 += 2) {
-          CodeVec cv[2];
+        for (int i = 0; i < kItersK; ++i) {
+          const int it = t + kKThreads * i;
+          if (it >= kItems) break;
+          const CodeVec cv = cv_next;
+          const int it_next = it + kKThreads;
+          if (it_next < kItems) cv_next = load_codes(it_next);
+          const int key = item_key<D>(it), blk = item_blk<D>(it);
+          uint32_t v[16];
+          if (key < valid) {
+            unpack_codes32(cv, v);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int it = t + kKThreads * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
-            if (i0 + i < kItersK && it < kItems)
-              cv[i] = *reinterpret_cast<const CodeVec*>(kcodes + key * (D * BITS / 8) + blk * (4 * BITS));
+            for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int it = t + kKThreads * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
-            if (i0 + i >= kItersK || it >= kItems) break;
-            uint32_t v[16];
-            if (key < valid) {
-              unpack_codes32(cv[i], v);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = 0u;
-            }
-            store32<N>(kt, key, blk, v);
-          }
+          store32<N>(kt, key, blk, v);
         }
         // Per-key constants of the tile: scales a for the softmax (once it has read the previous
         // ones from this buffer) and the key extras of the S MMA.
@@ -643,31 +643,32 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const uint8_t* vmeta = vcodes + C::kCodes;
         if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
         using CodeVec = typename CodeVecT<BITS>::type;
-        constexpr int kBatch = 2;                 // items per iteration; the loop is not unrolled
+        // One item per iteration with the next item's codes and (step, zero-point) already loaded
+        // (shared-memory loads are slow while the tensor core reads its operands); the loop itself
+        // is not unrolled.
+        struct VItem { CodeVec cv; float st, zp; };
+        auto load_item = [&](int it) {
+          VItem r;
+          const int key = item_key<D>(it), blk = item_blk<D>(it), g = (blk * 32) / C::G;
+          r.cv = *reinterpret_cast<const CodeVec*>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS));
+          if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, r.st, r.zp);
+          else load_meta<false>(vmeta, key * NG + g, r.st, r.zp);
+          return r;
+        };
+        VItem nxt = load_item(t);
 #pragma unroll 1
-        for (int i0 = 0; i0 < kItersV; i0 += kBatch) {
-          CodeVec cv[kBatch];
-          float st[kBatch], zp[kBatch];
+        for (int i = 0; i < kItersV; ++i) {
+          const int it = t + 128 * i, key = item_key<D>(it), blk = item_blk<D>(it);
+          const VItem cur = nxt;
+          if (i + 1 < kItersV) nxt = load_item(it + 128);
+          uint32_t v[16];
+          if (key < valid) {
+            dequant32(cur.cv, cur.st, cur.zp, v);
+          } else {
 #pragma unroll
-          for (int i = 0; i < kBatch; ++i) {
-            const int it = t + 128 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
-            const int g = (blk * 32) / C::G;
-            cv[i] = *reinterpret_cast<const CodeVec*>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS));
-            if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, st[i], zp[i]);
-            else load_meta<false>(vmeta, key * NG + g, st[i], zp[i]);
+            for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
-#pragma unroll
-          for (int i = 0; i < kBatch; ++i) {
-            const int it = t + 128 * (i0 + i), key = item_key<D>(it), blk = item_blk<D>(it);
-            uint32_t v[16];
-            if (key < valid) {
-              dequant32(cv[i], st[i], zp[i], v);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = 0u;
-            }
-            store32<N>(vt, key, blk, v);
-          }
+          store32<N>(vt, key, blk, v);
         }
         fence_async_smem();
         __syncwarp();
