@@ -25,6 +25,8 @@ Readings taken where the pages are silent (each one is also listed in the design
   * Score scale: s = scale * q.k with scale = 1/sqrt(d) unless given; the correction is in the
     same scaled-score units. For a general scale the Taylor term is (scale^2/24) sum_c q_c^2
     Delta_c^2, which is the page's (1/(24 d)) sum_c q_c^2 Delta_{i,c}^2 at scale = 1/sqrt(d).
+  * Correction modes: 0 none, 1 the second-order Taylor form of [JB] 方法, 2 the series of the exact
+    form to fourth order (a^2/6 - a^4/180 per channel), 3 the exact form (oracle only).
   * Exact correction (not printed on the pages, called numerically unfavourable in [JB] 方法):
     uniform rounding noise e_c ~ U(-Delta_c/2, Delta_c/2) gives E[e^{a u}] = sinh(a)/a, so
     b = sum_c log(sinh(a_c)/a_c), a_c = scale * q_c * Delta_c / 2.
@@ -45,7 +47,7 @@ import numpy as np
 __all__ = [
     "META_DTYPES", "levels", "quantize", "pack_codes", "unpack_codes", "dequantize",
     "build_cache", "cache_rows", "log_sinhc", "jensen_bias_taylor", "jensen_bias_exact",
-    "attention_rows", "corrected_attention", "merge_partials",
+    "attention_rows", "corrected_attention", "merge_partials", "jensen_bias_taylor4",
 ]
 
 META_DTYPES = {"f32": np.float32, "f16": np.float16}
@@ -176,6 +178,20 @@ def jensen_bias_taylor(q: np.ndarray, step: np.ndarray, group: int, scale: float
     return (scale * scale / 24.0) * ((q * q) @ (dc * dc).T)
 
 
+def jensen_bias_taylor4(q: np.ndarray, step: np.ndarray, group: int, scale: float) -> np.ndarray:
+    """Correction to fourth order: b_ij = sum_c (a^2/6 - a^4/180), a = scale q_ic Delta_{j,c} / 2.
+
+    The first two terms of the series of log(sinh a / a) (the exact form below). The a^2 term is
+    the second-order correction of [JB] 方法; the a^4 term is
+    -(scale^4 / 2880) sum_c q_ic^4 Delta_{j,c}^4, again a sum over channel groups of a per-query
+    power sum times a per-key step power.
+    """
+    dc = _per_channel(step, group)
+    q = np.asarray(q, dtype=np.float64)
+    q2 = q * q
+    return jensen_bias_taylor(q, step, group, scale) - (scale ** 4 / 2880.0) * ((q2 * q2) @ (dc ** 4).T)
+
+
 def jensen_bias_exact(q: np.ndarray, step: np.ndarray, group: int, scale: float) -> np.ndarray:
     """Exact correction for uniform rounding noise: b_ij = sum_c log(sinh(a)/a), a = scale q_ic Delta_{j,c} / 2."""
     dc = _per_channel(step, group)
@@ -198,7 +214,7 @@ def attention_rows(q: np.ndarray, q_pos: np.ndarray, k_hat: np.ndarray, v_hat: n
     """Attention of query rows q [n, d] (positions q_pos in the chunk of Lq queries).
 
     k_hat, v_hat [Lc, d]: dequantised cache; k_step [Lc, n_g]; k_cur, v_cur [Lcur, d].
-    correct: 0 none, 1 Taylor (the paper's), 2 exact (oracle only).
+    correct: 0 none, 1 second-order Taylor (the paper's), 2 fourth-order Taylor, 3 exact (oracle only).
     Returns O [n, d] and LSE [n] (natural log), fp64.
     """
     q = np.asarray(q, dtype=np.float64)
@@ -209,6 +225,8 @@ def attention_rows(q: np.ndarray, q_pos: np.ndarray, k_hat: np.ndarray, v_hat: n
     if correct == 1 and Lc:
         s_cache = s_cache - jensen_bias_taylor(q, k_step, group, scale)
     elif correct == 2 and Lc:
+        s_cache = s_cache - jensen_bias_taylor4(q, k_step, group, scale)
+    elif correct == 3 and Lc:
         s_cache = s_cache - jensen_bias_exact(q, k_step, group, scale)
     s_cur = scale * (q @ k_cur.T)
     if causal and Lcur:

@@ -5,6 +5,7 @@ b_i = log E[exp(delta_i)] with delta_i the score error of cached key i (agents-r
 """
 import json
 import math
+from fractions import Fraction
 import os
 
 import mpmath
@@ -142,3 +143,67 @@ def test_bias_scaling_and_zero():
     np.testing.assert_allclose(b3, 9.0 * b1, rtol=1e-13)
     assert np.all(oracle.jensen_bias_taylor(q, np.zeros((7, 2)), 16, 0.3) == 0)
     assert np.all(oracle.jensen_bias_exact(q, np.zeros((7, 2)), 16, 0.3) == 0)
+
+
+# --------------------------------------------------------------------------------------------
+# Fourth-order correction (the a^4 term of the series of log(sinh a / a)).
+# --------------------------------------------------------------------------------------------
+def test_taylor4_worked_example():
+    """One channel, q = 2, Delta = 1, scale = 0.5: a = scale q Delta / 2 = 0.5, so
+    b = a^2/6 - a^4/180 = 1/24 - 1/2880 = 119/2880 (by hand)."""
+    b = oracle.jensen_bias_taylor4(np.array([[2.0]]), np.array([[1.0]]), 1, 0.5)
+    assert b.shape == (1, 1)
+    assert abs(b[0, 0] - 119.0 / 2880.0) < 1e-15
+
+
+def test_taylor4_sums_the_channels_of_each_group():
+    """Channels of one group share the key's step: b = sum_c (a_c^2/6 - a_c^4/180), checked with
+    exact rationals channel by channel."""
+    q = np.array([[1.0, 2.0, 3.0, -1.5]])
+    step = np.array([[0.75, 1.25]])              # groups of 2 channels
+    scale = 0.5
+    want = Fraction(0)
+    for c, qc in enumerate(q[0]):
+        a = Fraction(scale) * Fraction(qc) * Fraction(step[0, c // 2]) / 2
+        want += a * a / 6 - a ** 4 / 180
+    got = oracle.jensen_bias_taylor4(q, step, 2, scale)[0, 0]
+    assert abs(got - float(want)) < 1e-15
+
+
+@pytest.mark.parametrize("a", [0.02, 0.05, 0.1, 0.2])
+def test_taylor4_error_against_mpmath_is_the_sixth_order_term(a):
+    """log(sinh a / a) = a^2/6 - a^4/180 + a^6/2835 - ...: the fourth-order form misses the exact
+    value by a^6/2835 to leading order (exact value from mpmath at 50 digits)."""
+    import mpmath
+    mpmath.mp.dps = 50
+    exact = float(mpmath.log(mpmath.sinh(a) / a))
+    b4 = oracle.jensen_bias_taylor4(np.array([[2.0 * a]]), np.array([[1.0]]), 1, 1.0)[0, 0]
+    b2 = oracle.jensen_bias_taylor(np.array([[2.0 * a]]), np.array([[1.0]]), 1, 1.0)[0, 0]
+    assert abs((exact - b4) / (a ** 6 / 2835.0) - 1.0) < 0.01 + 2 * a * a
+    assert abs(exact - b4) < abs(exact - b2)     # the extra term brings the form closer
+
+
+def test_taylor4_modes_in_attention():
+    """correct = 2 subtracts the fourth-order form, correct = 3 the exact one (oracle only)."""
+    rng = np.random.default_rng(3)
+    d, group, Lc, Lcur, Lq = 8, 4, 20, 5, 5
+    q = rng.normal(size=(Lq, d))
+    k_hat = rng.normal(size=(Lc, d))
+    v_hat = rng.normal(size=(Lc, d))
+    step = rng.uniform(0.2, 1.5, (Lc, d // group))
+    kc, vc = rng.normal(size=(Lcur, d)), rng.normal(size=(Lcur, d))
+    scale = 1 / math.sqrt(d)
+    outs = {}
+    for correct in (1, 2, 3):
+        outs[correct] = oracle.attention_rows(q, np.arange(Lq), k_hat, v_hat, step, group, kc, vc,
+                                              correct, False, scale, Lq)[1]
+    b2 = oracle.jensen_bias_taylor(q, step, group, scale)
+    b4 = oracle.jensen_bias_taylor4(q, step, group, scale)
+    s = scale * q @ k_hat.T
+    for correct, b in ((1, b2), (2, b4)):
+        s_all = np.concatenate([s - b, scale * q @ kc.T], axis=1)
+        lse = np.log(np.exp(s_all).sum(1))
+        np.testing.assert_allclose(outs[correct], lse, rtol=0, atol=1e-12)
+    # the fourth-order LSE lies between the second-order and the exact one (b2 >= b_exact, b4 <= b_exact
+    # for these small a, so LSE(b2) <= LSE(exact) <= LSE(b4))
+    assert np.all(outs[1] <= outs[3] + 1e-15) and np.all(outs[3] <= outs[2] + 1e-15)
