@@ -112,7 +112,11 @@ qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H
  *  Q            : dtype [B][H_q][L_q][d]; dtype QKV_F32 or QKV_BF16. H_q % H_kv == 0; query head
  *                 hq reads KV head hq / (H_q / H_kv).
  *  K_cur, V_cur : dtype [B][H_kv][L_cur][d], the unquantised current chunk (may be NULL if L_cur=0).
- *  correct      : 0 = plain attention over the dequantised cache, 1 = Taylor correction.
+ *  correct      : 0 = plain attention over the dequantised cache, 1 = Taylor correction (the
+ *                 summary's second-order form), 2 = the series of the exact correction
+ *                 sum_c log(sinh(a_c)/a_c), a_c = scale*q_c*step/2, to fourth order:
+ *                 b_j = sum_c (a_c^2/6 - a_c^4/180), i.e. the term above minus
+ *                 (scale^4 / 2880) * sum_c q_c^4 * step_{j, c/group}^4.
  *  causal_cur   : 1 = query i sees current key j only if j <= i + (L_cur - L_q); the cache is
  *                 always fully visible.
  *  scale        : score scale; <= 0 means 1/sqrt(d).

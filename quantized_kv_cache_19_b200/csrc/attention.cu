@@ -113,7 +113,7 @@ __host__ __device__ inline Layout make_layout(int meta_bytes) {
   L.vt = L.kt + 2 * C::kTile;
   L.pk = L.vt + 2 * C::kTile;
   L.kc = L.pk + C::kStages * L.stage;
-  L.ax = (L.kc + 2 * C::kKconst + 127) & ~127u;
+  L.ax = (L.kc + 4 * C::kKconst + 127) & ~127u;   // scales a (2 buffers), then step^4 (2 buffers)
   L.bx = L.ax + C::kAx;
   L.xc = L.bx + 2 * C::kBx;                // row-max exchange [2][2][128] and row-sum [2][128]
   L.bars = L.xc + (4 + 2) * kBM * 4;
@@ -366,7 +366,7 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int D, int BITS, int NG>
+template <int D, int BITS, int NG, bool kQuartic>
 __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const AttnParams p) {
   using C = Cfg<D, BITS, NG>;
   constexpr int N = C::N;
@@ -554,12 +554,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const uint8_t* kmeta = kcodes + C::kCodes;
         float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
         constexpr int kItersC = (N * NG + kKThreads - 1) / kKThreads;
-#pragma unroll
+#pragma unroll 1
         for (int i = 0; i < kItersC; ++i) {
           const int e = t + kKThreads * i;
           if (e >= N * NG) break;
           const int key = e / NG, g = e % NG;
-          float a = 0.f, rho = 0.f, sigma = 0.f;
+          float a = 0.f, rho = 0.f, sigma = 0.f, d4 = 0.f;
           if (key < valid) {
             float step, zp;
             if (p.meta_f16) load_meta<true>(kmeta, key * NG + g, step, zp);
@@ -568,8 +568,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
             a = sp * p.scale_log2;
             rho = zp / sp;
             sigma = step * p.inv_scale_log2;
+            const float s2 = step * step;
+            d4 = s2 * s2;                                 // fourth-order term (softmax, fp32)
           }
-          kc[((key >> 1) * C::NAH + (g >> 1)) * 4 + (g & 1) * 2 + (key & 1)] = a;
+          const int ci = ((key >> 1) * C::NAH + (g >> 1)) * 4 + (g & 1) * 2 + (key & 1);
+          kc[ci] = a;
+          kc[2 * (C::kKconst / 4) + ci] = d4;
           __nv_bfloat16 rh, rm, rl, sh, sm, sl;
           split3(rho, rh, rm, rl);
           split3(sigma, sh, sm, sl);
@@ -596,7 +600,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
         float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
 #pragma unroll 1
-        for (int e = t; e < static_cast<int>(C::kKconst / 4); e += kKThreads) kc[e] = p.scale_log2;
+        for (int e = t; e < static_cast<int>(C::kKconst / 4); e += kKThreads) {
+          kc[e] = p.scale_log2;
+          kc[2 * (C::kKconst / 4) + e] = 0.f;        // no correction on current keys
+        }
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(bar(B_KH_FULL + sb));
@@ -711,12 +718,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     // Q row: group sums of q (what the codes multiply), correction weights; this half's columns of
     // the bf16 copy of Q go into TMEM.
     float w[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
+    float u[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};   // fourth-order weights (correct = 2)
     float qs[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
     {
       const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * 2;
       uint32_t qp[D / 4];
       if (valid_row) {
-        query_group_weights<D>(qrow, false, C::G, p.wcoef_log2, w);
+        query_group_powers<D>(qrow, false, C::G, p.wcoef_log2, kQuartic ? p.ucoef_log2 : 0.f, w, u);
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) {
           float x[8];
@@ -741,9 +749,11 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       }
       tmem_st<D / 4>(tmem + lane_off + kColQ + half * (D / 4), qp);
       if (half == 0) {
-        // row extras per group [qs_h, qs_h, qs_m, qs_h, qs_m, qs_l, nw_h, nw_h, nw_m, nw_h, nw_l, nw_m, 0..]
-        // against the key extras [rho_h, rho_m, rho_h, rho_l, rho_m, rho_h, sig_h, sig_m, sig_h, sig_l,
-        // sig_h, sig_m, 0..]: every product of parts whose orders add up to at most two.
+        // row extras per group [qs_h, qs_h, qs_m, qs_h, qs_m, qs_l, nw_h, nw_h, nw_m, nw_h, nw_l, nw_m,
+        // 0..] against the key extras [rho_h, rho_m, rho_h, rho_l, rho_m, rho_h, sig_h, sig_m, sig_h,
+        // sig_l, sig_h, sig_m, 0..]: every product of parts whose orders add up to at most two. The
+        // fourth-order term (correct = 2) is added in the softmax in fp32 instead: for keys with
+        // large steps its series term grows without bound, beyond what bf16 parts resolve.
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
           __nv_bfloat16 qh, qm, ql, nh, nm, nl;
@@ -765,6 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       for (int g = 0; g < kMaxGroups; ++g) w[g] = 0.f;
     }
 
+    constexpr bool quartic = kQuartic;   // correct = 2: fourth-order term in the softmax
     float m_run = -INFINITY;   // max used for the exponentials so far (log2 units), same in both halves
     float l_run = 0.f;         // this half's part of the softmax denominator
     const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
@@ -795,6 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       if (!warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
       // s = sum_g a_g * S_g: per-key group scales for cached tiles, the score scale for current ones.
       const float4* ka = kconst + kb * (C::kKconst / 16);
+      const float4* kd4 = kconst + (2 + kb) * (C::kKconst / 16);
 #pragma unroll
       for (int c0 = 0; c0 < NH; c0 += kCK) {
         uint32_t r[C::NA][kCK];
@@ -814,6 +826,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
               acc = __ffma2_rn(make_float2(a.z, a.w),
                                make_float2(__uint_as_float(r[2 * ah + 1][2 * q]),
                                            __uint_as_float(r[2 * ah + 1][2 * q + 1])), acc);
+            if (quartic) {                          // + u_g * step_g^4 (fourth-order term)
+              const float4 d = kd4[pq * C::NAH + ah];
+              acc = __ffma2_rn(make_float2(d.x, d.y), make_float2(u[2 * ah], u[2 * ah]), acc);
+              if (2 * ah + 1 < C::NA)
+                acc = __ffma2_rn(make_float2(d.z, d.w), make_float2(u[2 * ah + 1], u[2 * ah + 1]), acc);
+            }
           }
           s2[c0 / 2 + q] = acc;
         }
@@ -955,29 +973,30 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
   }
 }
 
-template <int D, int BITS, int NG>
+template <int D, int BITS, int NG, bool kQuartic>
 cudaError_t launch_impl(const AttnParams& p, cudaStream_t stream) {
   const Layout L = make_layout<D, BITS, NG>(p.meta_f16 ? 2 : 4);
   // At least 116 KB so that two CTAs never share an SM: each holds all 512 TMEM columns.
   size_t smem = L.total + 1024;
   if (smem < 116u * 1024u) smem = 116u * 1024u;
-  cudaError_t e = cudaFuncSetAttribute(corrected_attention_kernel<D, BITS, NG>,
+  cudaError_t e = cudaFuncSetAttribute(corrected_attention_kernel<D, BITS, NG, kQuartic>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(p.r) * p.Lq;
   dim3 grid(static_cast<unsigned>((rows + kBM - 1) / kBM), static_cast<unsigned>(p.B * p.Hkv),
             static_cast<unsigned>(p.n_split > 1 ? p.n_split : 1));
-  corrected_attention_kernel<D, BITS, NG><<<grid, kThreads, smem, stream>>>(p);
+  corrected_attention_kernel<D, BITS, NG, kQuartic><<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 template <int D, int BITS>
 cudaError_t launch_groups(const AttnParams& p, cudaStream_t stream) {
-  if (p.n_groups == 1) return launch_impl<D, BITS, 1>(p, stream);
-  if (p.n_groups == 2) return launch_impl<D, BITS, 2>(p, stream);
+  const bool q4 = p.correct == 2;
+  if (p.n_groups == 1) return q4 ? launch_impl<D, BITS, 1, true>(p, stream) : launch_impl<D, BITS, 1, false>(p, stream);
+  if (p.n_groups == 2) return q4 ? launch_impl<D, BITS, 2, true>(p, stream) : launch_impl<D, BITS, 2, false>(p, stream);
   if constexpr (D == 128) {
-    if (p.n_groups == 4) return launch_impl<D, BITS, 4>(p, stream);
+    if (p.n_groups == 4) return q4 ? launch_impl<D, BITS, 4, true>(p, stream) : launch_impl<D, BITS, 4, false>(p, stream);
   }
   return cudaErrorInvalidValue;
 }

@@ -48,9 +48,10 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
   const int row_codes = D * bits / 8;
 
   float w[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
+  float u[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
   const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * 4;
   if (valid_row) {
-    if (p.correct) query_group_weights<D>(qrow, true, G, wcoef, w);
+    if (p.correct) query_group_powers<D>(qrow, true, G, wcoef, p.ucoef_log2 * 0.69314718055994530942f, w, u);
     for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = reinterpret_cast<const float*>(qrow)[c];
   } else {
     for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = 0.f;
@@ -106,6 +107,9 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
         float d2[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
         for (int g = 0; g < NG; ++g) d2[g] = d2_s[kk * 4 + g];
         s -= jensen_term(w, d2, NG);
+        if (p.correct == 2) {
+          for (int g = 0; g < NG; ++g) s = fmaf(u[g], d2[g] * d2[g], s);
+        }
       }
       if (s > m) {
         const float a = expf(m - s);       // 0 when m = -inf

@@ -202,7 +202,7 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
     return fail(QKV_ERR_INVALID_ARG, "H_q %d must be a positive multiple of H_kv %d", H_q,
                 cache->H_kv);
   if (L_q < 0 || L_cur < 0) return fail(QKV_ERR_INVALID_ARG, "negative length");
-  if (correct != 0 && correct != 1) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0 or 1");
+  if (correct < 0 || correct > 2) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0, 1 or 2");
   if (causal_cur != 0 && causal_cur != 1) return fail(QKV_ERR_INVALID_ARG, "causal_cur must be 0 or 1");
   if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
   if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
@@ -232,6 +232,7 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   p.scale_log2 = sc * log2e;
   p.wcoef_log2 = sc * sc / 24.0f * log2e;
   p.inv_scale_log2 = 1.0f / (sc * log2e);
+  p.ucoef_log2 = correct == 2 ? sc * sc * sc * sc / 2880.0f * log2e : 0.0f;
   p.n_split = 1;
   p.rows_all = static_cast<int64_t>(cache->B) * H_q * L_q;
   p.ws_o = nullptr;
@@ -354,7 +355,7 @@ QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int
     return fail(QKV_ERR_INVALID_ARG, "H_q %d must be a positive multiple of H_kv %d", H_q,
                 cache->H_kv);
   if (L_q < 0 || L_cur < 0) return fail(QKV_ERR_INVALID_ARG, "negative length");
-  if (correct != 0 && correct != 1) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0 or 1");
+  if (correct < 0 || correct > 2) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0, 1 or 2");
   if (causal_cur != 0 && causal_cur != 1) return fail(QKV_ERR_INVALID_ARG, "causal_cur must be 0 or 1");
   if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
   if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
@@ -397,6 +398,7 @@ QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int
   p.scale_log2 = sc * log2e;
   p.wcoef_log2 = sc * sc / 24.0f * log2e;
   p.inv_scale_log2 = 1.0f / (sc * log2e);
+  p.ucoef_log2 = correct == 2 ? sc * sc * sc * sc / 2880.0f * log2e : 0.0f;
   p.n_split = n;
   p.rows_all = static_cast<int64_t>(cache->B) * H_q * L_q;
   p.ws_o = scratch;

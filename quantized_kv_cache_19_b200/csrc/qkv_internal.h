@@ -46,6 +46,7 @@ struct AttnParams {
   float scale_log2;   // score scale * log2(e)
   float wcoef_log2;   // scale^2 / 24 * log2(e): Jensen-correction coefficient in log2 units
   float inv_scale_log2;  // 1 / (scale * log2(e))
+  float ucoef_log2;   // scale^4 / 2880 * log2(e): fourth-order coefficient (correct = 2), else 0
   // Split over the cached keys (n_split > 1): CTA z takes cached tiles [z * T / n, (z+1) * T / n)
   // (the last one also the current chunk) and writes its row's normalised partial output and
   // log-sum-exp to ws_o [n_split][rows_all][d] and ws_lse [n_split][rows_all] (fp32).

@@ -47,6 +47,35 @@ __device__ __forceinline__ void query_group_weights(const uint8_t* qrow, bool f3
   for (int g = 0; g < kMaxGroups; ++g) w[g] *= coef;
 }
 
+// Second- and fourth-order weights in one pass over the row: w[g] = coef2 * sum_{c in g} q_c^2 and
+// u[g] = coef4 * sum_{c in g} q_c^4 (the a^4 / 180 term of the series of log(sinh a / a),
+// a = scale q_c Delta / 2, is (scale^4 / 2880) q_c^4 Delta^4).
+template <int D>
+__device__ __forceinline__ void query_group_powers(const uint8_t* qrow, bool f32, int group, float coef2,
+                                                   float coef4, float (&w)[kMaxGroups],
+                                                   float (&u)[kMaxGroups]) {
+#pragma unroll
+  for (int g = 0; g < kMaxGroups; ++g) { w[g] = 0.f; u[g] = 0.f; }
+#pragma unroll
+  for (int c8 = 0; c8 < D / 8; ++c8) {
+    float x[8];
+    load_q8(qrow, f32, c8, x);
+    float a2 = 0.f, a4 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float x2 = x[k] * x[k];
+      a2 += x2;
+      a4 = fmaf(x2, x2, a4);
+    }
+    const int g = (c8 * 8) / group;
+#pragma unroll
+    for (int gg = 0; gg < kMaxGroups; ++gg)
+      if (gg == g) { w[gg] += a2; u[gg] += a4; }
+  }
+#pragma unroll
+  for (int g = 0; g < kMaxGroups; ++g) { w[g] *= coef2; u[g] *= coef4; }
+}
+
 // The correction of one (query, key) pair from the key's squared steps: sum_g w[g] * d2[g].
 __device__ __forceinline__ float jensen_term(const float (&w)[kMaxGroups],
                                              const float (&d2)[kMaxGroups], int n_groups) {

@@ -16,13 +16,13 @@ from parity_utils import (BIAS_REL_TOL, build_gpu_cache, check_full, check_sampl
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("correct", [0, 1])
+@pytest.mark.parametrize("correct", [0, 1, 2])
 @pytest.mark.parametrize("name", ["tiny_f32", "bf16_int4", "bf16_int2"])
 def test_small_workloads_every_row(name, correct):
     check_full(WORKLOADS[name], correct)
 
 
-@pytest.mark.parametrize("correct", [0, 1])
+@pytest.mark.parametrize("correct", [0, 1, 2])
 @pytest.mark.parametrize("name,heads", [
     ("video_dit", [(0, 0), (0, 11), (0, 23)]),
     ("long_video", [(0, 0), (0, 39)]),
@@ -50,7 +50,7 @@ EDGE = {
 }
 
 
-@pytest.mark.parametrize("correct", [0, 1])
+@pytest.mark.parametrize("correct", [0, 1, 2])
 @pytest.mark.parametrize("case", sorted(EDGE))
 def test_edge_cases(case, correct):
     base = WORKLOADS["bf16_int2"].with_(Hq=2, Hkv=2, Lq=64, Lcur=64, Lc=256, seed=77)
@@ -94,3 +94,21 @@ def test_repeated_calls_are_deterministic():
     O2, L2 = api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1)
     torch.cuda.synchronize()
     assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_fourth_order_term_is_applied(dtype):
+    """correct = 2 matches the oracle's fourth-order form and differs from the second-order one by
+    far more than the tolerance on keys with outlier channels (large steps)."""
+    w = WORKLOADS["bf16_int2"].with_(Hq=2, Hkv=2, Lq=64, Lcur=64, Lc=512, dtype=dtype, seed=78)
+    x = make_inputs(w, device="cuda")
+    cache = build_gpu_cache(w, x["K_src"], x["V_src"])
+    O, L = api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=2)
+    torch.cuda.synchronize()
+    sub = sub_problem(x, w, 0, 1)
+    O4, L4 = oracle_head(w, sub, 2)
+    O2, L2 = oracle_head(w, sub, 1)
+    Lg = np32(L[0:1, 1:2]).astype(np.float64)
+    compare(np32(O[0:1, 1:2]).astype(np.float64), O4, Lg, L4, f"fourth order {dtype}")
+    assert np.max(np.abs(L4 - L2)) > 10 * 2e-3
+    assert api.device_status() == 0

@@ -86,7 +86,8 @@ def test_attention_rejections(lib):
     c2 = _fake_cache(length=100)
     assert call(c=c2, Hq=3) == api.QKV_ERR_INVALID_ARG               # H_q not a multiple of H_kv
     assert call(c=c2, dt=api.QKV_F16) == api.QKV_ERR_UNSUPPORTED
-    assert call(c=c2, corr=2) == api.QKV_ERR_UNSUPPORTED             # exact correction is oracle-only
+    assert call(c=c2, corr=3) == api.QKV_ERR_UNSUPPORTED             # exact correction is oracle-only
+    assert call(c=c2, corr=-1) == api.QKV_ERR_UNSUPPORTED
     assert call(c=c2, Q=P(0x70002)) == api.QKV_ERR_INVALID_ARG       # misaligned
     assert call(c=c2, Lcur=8, K=None) == api.QKV_ERR_INVALID_ARG
     assert call(c=c2, scale=float("nan")) == api.QKV_ERR_INVALID_ARG

@@ -18,7 +18,7 @@ def _decode(Lq, **kw):
 
 
 @pytest.mark.parametrize("Lq", [1, 4, 16])
-@pytest.mark.parametrize("correct", [0, 1])
+@pytest.mark.parametrize("correct", [0, 1, 2])
 def test_split_keys_every_row(Lq, correct):
     w = _decode(Lq)
     cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc), w.meta)
