@@ -12,7 +12,11 @@ Sources (cited by page title and section):
          subtract b_i from quantised-key scores before the softmax), 「限制與邊界情況」 (limits).
   [ABS]  fugumt.com, "Quantized Keys Steal Attention: Bias Correction for KV-Cache Compression
          in Video Diffusion", Abstract (correction from step sizes and query norm, no extra memory).
-  [QWM]  pchao.org, "QuantWM：保住时间一致性的两比特键值缓存量化", eq. (5): logits are Q K^T / sqrt(d).
+  [QWM]  pchao.org, "QuantWM：保住时间一致性的两比特键值缓存量化", eq. (5): logits are Q K^T / sqrt(d);
+         section 实验如何设计 (token drift: top-1 attended token differing from the BF16 one).
+  [SIQ]  gist.science, "Statistical Inference and Quality Measures of KV Cache Quantisations
+         Inspired by TurboQuant", section Métricas de Avaliação (KL divergence between reference and
+         quantised softmax distributions, top-5 recall).
 
 Readings taken where the pages are silent (each one is also listed in the design notes):
   * Quantiser: asymmetric min-max per (token, head, group of `group` consecutive channels);
@@ -36,6 +40,10 @@ Readings taken where the pages are silent (each one is also listed in the design
     (of Lq) sees current key j (of Lcur) iff j <= i + (Lcur - Lq). The cache is always visible.
   * GQA: query head hq reads KV head hq // (Hq // Hkv).
   * LSE is the natural-log log-sum-exp of the corrected scores of each query row.
+  * Fidelity diagnostics: the reference distribution is the softmax over the cached keys as they
+    were before quantisation (in the input precision) and the current keys; the quantised one is
+    the corrected attention's softmax. Top-k lists break equal scores by the lower key index;
+    recall counts over min(k, visible keys) keys; the top-k size is 5 ([SIQ]).
 """
 from __future__ import annotations
 
@@ -48,6 +56,7 @@ __all__ = [
     "META_DTYPES", "levels", "quantize", "pack_codes", "unpack_codes", "dequantize",
     "build_cache", "cache_rows", "log_sinhc", "jensen_bias_taylor", "jensen_bias_exact",
     "attention_rows", "corrected_attention", "merge_partials", "jensen_bias_taylor4",
+    "FIDELITY_TOPK", "fidelity_rows",
 ]
 
 META_DTYPES = {"f32": np.float32, "f16": np.float16}
@@ -298,3 +307,86 @@ def merge_partials(parts: Sequence[Tuple[np.ndarray, np.ndarray]]) -> Tuple[np.n
     lse = m + np.log(w.sum(axis=0))
     o = sum(np.exp(p[1] - lse)[..., None] * p[0] for p in parts)
     return o, lse
+
+
+# --------------------------------------------------------------------------------------------
+# Attention-fidelity diagnostics: how far the softmax over the quantised cache is from the one
+# over the unquantised keys. [QWM] 实验如何设计 defines the token drift rate as the share of
+# positions whose top-1 attended token under the quantised cache differs from the BF16 one;
+# [SIQ] Métricas de Avaliação uses the KL divergence between the reference and the quantised
+# softmax distributions and the recall of the reference's top-5 keys; [JB] 為何校正有效 and the
+# [ABS] title describe the quantised keys' excess ("stolen") attention mass on the cached segment.
+# --------------------------------------------------------------------------------------------
+FIDELITY_TOPK = 5
+
+
+def _top_keys(s: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest finite scores of each row, largest first, the lower index first on
+    equal scores; -1 where a row has fewer than k visible keys."""
+    n = s.shape[0]
+    out = np.full((n, k), -1, dtype=np.int64)
+    for i in range(n):
+        vis = np.flatnonzero(np.isfinite(s[i]))
+        order = vis[np.argsort(-s[i, vis], kind="stable")]
+        out[i, :min(k, order.size)] = order[:k]
+    return out
+
+
+def fidelity_rows(q: np.ndarray, q_pos: np.ndarray, k_ref: np.ndarray, k_hat: np.ndarray,
+                  k_step: np.ndarray, group: int, k_cur: np.ndarray, correct: int, causal: bool,
+                  scale: float, Lq: int, topk: int = FIDELITY_TOPK) -> Dict[str, np.ndarray]:
+    """Per query row q [n, d] (positions q_pos in the chunk of Lq queries), fp64:
+
+    P_ref: softmax of scale q.k over [k_ref ; k_cur] (k_ref [Lc, d]: the cached keys unquantised);
+    P_q:   softmax over [k_hat ; k_cur] of scale q.k minus the correction of mode `correct` on the
+           cached keys (the scores of `attention_rows`).
+    Returns lse_ref, lse_q (natural log), mass_ref, mass_q (total probability of the Lc cached keys),
+    kl = KL(P_ref || P_q) = sum_j P_ref,j (log P_ref,j - log P_q,j), top_ref / top_q [n, topk] (the
+    `_top_keys` of each score row; key index j < Lc is cached key j, Lc + t is current key t),
+    top1_agree (1.0 where the two top-1 keys coincide) and recall (share of the reference's top
+    keys that are among the quantised ones, over min(topk, visible keys) keys).
+    A row that sees no key: lse -inf, masses 0, kl 0, top -1, top1_agree 1, recall 1.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_ref = np.asarray(k_ref, dtype=np.float64)
+    k_cur = np.asarray(k_cur, dtype=np.float64)
+    n, Lc, Lcur = q.shape[0], k_hat.shape[0], k_cur.shape[0]
+    s_ref_cache = scale * (q @ k_ref.T)
+    s_q_cache = scale * (q @ k_hat.T)
+    if correct == 1 and Lc:
+        s_q_cache = s_q_cache - jensen_bias_taylor(q, k_step, group, scale)
+    elif correct == 2 and Lc:
+        s_q_cache = s_q_cache - jensen_bias_taylor4(q, k_step, group, scale)
+    elif correct == 3 and Lc:
+        s_q_cache = s_q_cache - jensen_bias_exact(q, k_step, group, scale)
+    s_cur = scale * (q @ k_cur.T)
+    if causal and Lcur:
+        lim = np.asarray(q_pos)[:, None] + (Lcur - Lq)
+        s_cur = np.where(np.arange(Lcur)[None, :] <= lim, s_cur, -np.inf)
+    s_ref = np.concatenate([s_ref_cache, s_cur], axis=1)
+    s_q = np.concatenate([s_q_cache, s_cur], axis=1)
+
+    def log_softmax(s):
+        m = s.max(axis=1, initial=-np.inf)
+        m_safe = np.where(np.isfinite(m), m, 0.0)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            lse = m_safe + np.log(np.exp(s - m_safe[:, None]).sum(axis=1))
+            return s - lse[:, None], lse
+
+    logp_ref, lse_ref = log_softmax(s_ref)
+    logp_q, lse_q = log_softmax(s_q)
+    p_ref, p_q = np.exp(logp_ref), np.exp(logp_q)
+    vis = np.isfinite(s_ref)
+    kl = np.where(vis, p_ref * (np.where(vis, logp_ref, 0.0) - np.where(vis, logp_q, 0.0)), 0.0).sum(axis=1)
+    top_ref = _top_keys(s_ref, topk)
+    top_q = _top_keys(s_q, topk)
+    agree = np.ones(n)
+    recall = np.ones(n)
+    for i in range(n):
+        r = top_ref[i][top_ref[i] >= 0]
+        if r.size:
+            agree[i] = float(top_ref[i, 0] == top_q[i, 0])
+            recall[i] = np.isin(r, top_q[i]).sum() / r.size
+    return {"lse_ref": lse_ref, "lse_q": lse_q,
+            "mass_ref": p_ref[:, :Lc].sum(axis=1), "mass_q": p_q[:, :Lc].sum(axis=1),
+            "kl": kl, "top_ref": top_ref, "top_q": top_q, "top1_agree": agree, "recall": recall}
