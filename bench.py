@@ -51,6 +51,7 @@ CSRC = os.path.join(ROOT, "quantized_kv_cache_19_b200", "csrc")
 KERNEL_SOURCES = {
     "corrected_attention_kernel": ["attention.cu", "qkv_common.cuh", "qkv_jensen.cuh", "qkv_internal.h"],
     "quantize_append_kernel": ["quant_append.cu", "qkv_common.cuh", "qkv_internal.h"],
+    "attention_fidelity_kernel": ["fidelity.cu", "fidelity.h", "qkv_common.cuh", "qkv_jensen.cuh"],
 }
 
 
@@ -268,6 +269,46 @@ def decode_sweep(dev, peaks, flush, steps: int = 20):
     return out
 
 
+def fidelity_leg(w, x, cache, dev, flush, steps: int = 10):
+    """Attention-fidelity diagnostics (cached mass, KL, top-1 agreement, top-5 recall) over the
+    bench workload, correct=1, top lists written. fp32 CUDA-core arithmetic: 4d FLOP per (query row,
+    cached key) pair (two dot products) and 2d per visible current key, against the fp32 FMA peak
+    148 SMs x 128 lanes x 2 FLOP x the maximum SM clock."""
+    props = torch.cuda.get_device_properties(dev)
+    sm_mhz = float(load_peaks()[0].get("sm_max_mhz", 1965.0))
+    peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+    rows = w.B * w.Hq * w.Lq
+    if w.causal:
+        vis_cur = sum(max(0, min(w.Lcur, i + (w.Lcur - w.Lq) + 1)) for i in range(w.Lq)) * w.B * w.Hq
+    else:
+        vis_cur = rows * w.Lcur
+    flops = 4 * w.d * rows * w.Lc + 2 * w.d * vis_cur
+    stream = torch.cuda.current_stream(dev)
+    cache.length = w.Lc                      # the cache holds the quantised K_src in positions [0, Lc)
+    ts = []
+    for i in range(steps + 3):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        st, top = api.attention_fidelity(x["Q"], cache, x["K_src"], x["K_cur"], correct=1, causal=w.causal)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            ts.append(a.elapsed_time(b))
+    if api.device_status() != 0:
+        raise RuntimeError("device status after the fidelity diagnostics")
+    ms = statistics.mean(ts)
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"kernel": "attention_fidelity_kernel", "bound": "alu", "ms_per_launch": round(ms, 4),
+            "flops_per_launch": flops, "achieved": round(tf, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x max SM clock", "frac": round(tf / peak, 4),
+            "traffic": ncu_traffic("attention_fidelity_kernel", w.name),
+            "means": {"mass_ref": round(st[..., 2].mean().item(), 5), "mass_q": round(st[..., 3].mean().item(), 5),
+                      "kl": round(st[..., 4].mean().item(), 5),
+                      "token_drift": round(1.0 - st[..., 5].mean().item(), 5),
+                      "top5_recall": round(st[..., 6].mean().item(), 5)}}
+
+
 def run_ours(args, world, rank, local):
     w = WORKLOADS[args.workload]
     torch.cuda.set_device(local)
@@ -411,6 +452,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 2 * K,
         "clocks": clocks.summary(),
     }
+    if not args.no_fidelity:
+        result["fidelity"] = fidelity_leg(w, x, cache, dev, flush)
     if not args.no_decode:
         result["decode"] = decode_sweep(dev, peaks, flush)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -455,6 +498,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the few-query-rows (decode) sweep")
+    ap.add_argument("--no-fidelity", action="store_true", help="skip the attention-fidelity diagnostics")
     ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
                     help="store the DRAM bytes per launch of an ncu report (taken on --workload) and exit")
     ap.add_argument("--record-command", default="", help="the command line that made the report")

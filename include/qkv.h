@@ -162,6 +162,33 @@ qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, int64_t L_
                            const qkv_cache* cache, float scale, float* bias, void* stream);
 
 /*
+ * Attention-fidelity diagnostics: per query row, how far the corrected softmax over the quantised
+ * cache is from the softmax over the same keys before quantisation.
+ *   Token drift: pchao.org, "QuantWM：保住时间一致性的两比特键值缓存量化", section 实验如何设计
+ *   (share of positions whose top-1 attended token differs from the BF16 one).
+ *   KL and top-5 recall: gist.science, "Statistical Inference and Quality Measures of KV Cache
+ *   Quantisations Inspired by TurboQuant", section Métricas de Avaliação.
+ *   Cached mass: agents-report.net, "KV-Cache 量化導致的 Jensen 偏差", section 為何校正有效.
+ * P_ref is the softmax of scale * q.k over [K_ref ; K_cur]; P_q is corrected_attention's softmax
+ * (the same Q, cache, K_cur, correct, causal_cur and scale). V is not involved.
+ *  K_ref  : dtype [B][H_kv][cache->length][d], the cached keys as they were before quantisation
+ *           (may be NULL when cache->length = 0).
+ *  stats  : fp32 [B][H_q][L_q][8] = { LSE_ref, LSE_q, cached mass under P_ref, cached mass under
+ *           P_q, KL(P_ref || P_q), top-1 agreement (1 or 0), top-5 recall, 0 }. A row that sees no
+ *           key gets LSE -inf, masses and KL 0, agreement and recall 1.
+ *  top    : int32 [B][H_q][L_q][2][5] or NULL: the five highest-scoring keys of P_ref, then of
+ *           P_q, highest first, the lower index first on equal scores; key j < length is cached
+ *           key j, length + t is current key t; -1 pads rows that see fewer than 5 keys. Recall
+ *           counts the reference list's keys found in the quantised list, over min(5, keys seen).
+ * Every score is fp32 (CUDA cores). Pointers are device pointers, 16-byte aligned, caller-owned;
+ * nothing is allocated. length + L_cur must be below 2^31 - 1. Errors as corrected_attention.
+ */
+qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                              const qkv_cache* cache, const void* K_ref, const void* K_cur,
+                              int64_t L_cur, int32_t correct, int32_t causal_cur, float scale,
+                              float* stats, int32_t* top, void* stream);
+
+/*
  * Reads the library's device status word (0 = no error, else a qkv_status such as
  * QKV_ERR_TIMEOUT) into *code; clears it when reset != 0. Synchronises the current device.
  */

@@ -334,7 +334,8 @@ def _top_keys(s: np.ndarray, k: int) -> np.ndarray:
 
 def fidelity_rows(q: np.ndarray, q_pos: np.ndarray, k_ref: np.ndarray, k_hat: np.ndarray,
                   k_step: np.ndarray, group: int, k_cur: np.ndarray, correct: int, causal: bool,
-                  scale: float, Lq: int, topk: int = FIDELITY_TOPK) -> Dict[str, np.ndarray]:
+                  scale: float, Lq: int, topk: int = FIDELITY_TOPK,
+                  return_scores: bool = False) -> Dict[str, np.ndarray]:
     """Per query row q [n, d] (positions q_pos in the chunk of Lq queries), fp64:
 
     P_ref: softmax of scale q.k over [k_ref ; k_cur] (k_ref [Lc, d]: the cached keys unquantised);
@@ -346,6 +347,7 @@ def fidelity_rows(q: np.ndarray, q_pos: np.ndarray, k_ref: np.ndarray, k_hat: np
     top1_agree (1.0 where the two top-1 keys coincide) and recall (share of the reference's top
     keys that are among the quantised ones, over min(topk, visible keys) keys).
     A row that sees no key: lse -inf, masses 0, kl 0, top -1, top1_agree 1, recall 1.
+    With return_scores, also s_ref and s_q [n, Lc + Lcur] (-inf where a key is masked).
     """
     q = np.asarray(q, dtype=np.float64)
     k_ref = np.asarray(k_ref, dtype=np.float64)
@@ -387,6 +389,9 @@ def fidelity_rows(q: np.ndarray, q_pos: np.ndarray, k_ref: np.ndarray, k_hat: np
         if r.size:
             agree[i] = float(top_ref[i, 0] == top_q[i, 0])
             recall[i] = np.isin(r, top_q[i]).sum() / r.size
-    return {"lse_ref": lse_ref, "lse_q": lse_q,
-            "mass_ref": p_ref[:, :Lc].sum(axis=1), "mass_q": p_q[:, :Lc].sum(axis=1),
-            "kl": kl, "top_ref": top_ref, "top_q": top_q, "top1_agree": agree, "recall": recall}
+    out = {"lse_ref": lse_ref, "lse_q": lse_q,
+           "mass_ref": p_ref[:, :Lc].sum(axis=1), "mass_q": p_q[:, :Lc].sum(axis=1),
+           "kl": kl, "top_ref": top_ref, "top_q": top_q, "top1_agree": agree, "recall": recall}
+    if return_scores:
+        out["s_ref"], out["s_q"] = s_ref, s_q
+    return out

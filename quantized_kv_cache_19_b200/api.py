@@ -64,6 +64,9 @@ _SIGS = {
                                                    _P]),
     "qkv_jensen_bias": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
                                        ctypes.POINTER(QkvCacheDesc), ctypes.c_float, _P, _P]),
+    "attention_fidelity": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
+                                          ctypes.POINTER(QkvCacheDesc), _P, _P, ctypes.c_int64,
+                                          ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "qkv_device_status": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
 }
 
@@ -241,6 +244,37 @@ def attention_workspace_bytes(cache: KVCache, Hq: int, Lq: int, Lcur: int) -> in
     ws = ctypes.c_size_t()
     _check(lib.corrected_attention_workspace_bytes(ctypes.byref(cache.desc), Hq, Lq, Lcur, ctypes.byref(ws)))
     return int(ws.value)
+
+
+FIDELITY_FIELDS = ("lse_ref", "lse_q", "mass_ref", "mass_q", "kl", "top1_agree", "recall")
+
+
+def attention_fidelity(Q: torch.Tensor, cache: KVCache, K_ref: Optional[torch.Tensor],
+                       K_cur: Optional[torch.Tensor], correct: int = 1, causal: bool = False,
+                       scale: float = 0.0, with_top: bool = True
+                       ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Per-row fidelity of the quantised attention against the unquantised keys.
+
+    K_ref [B][H_kv][cache.length][d] (Q's dtype): the cached keys before quantisation.
+    Returns stats fp32 [B][H_q][L_q][8] (columns named by FIDELITY_FIELDS, the last one 0) and, with
+    with_top, top int32 [B][H_q][L_q][2][5]: the reference's and the quantised softmax's five
+    highest-scoring key indices (cached keys first, then current keys; -1 pads).
+    """
+    _need_cuda(Q, K_ref, K_cur)
+    B, Hq, Lq, d = Q.shape
+    Lcur = 0 if K_cur is None else K_cur.shape[2]
+    for t in (K_ref, K_cur):
+        if t is not None and t.dtype != Q.dtype:
+            raise ValueError("K_ref, K_cur must have Q's dtype")
+    if K_ref is not None and tuple(K_ref.shape) != (B, cache.H_kv, cache.length, d):
+        raise ValueError("K_ref must be [B][H_kv][cache.length][d]")
+    stats = torch.empty(B, Hq, Lq, 8, dtype=torch.float32, device=Q.device)
+    top = torch.empty(B, Hq, Lq, 2, 5, dtype=torch.int32, device=Q.device) if with_top else None
+    lib = load_library()
+    _check(lib.attention_fidelity(_ptr(Q), _DTYPE[Q.dtype], Hq, Lq, ctypes.byref(cache.desc),
+                                  _ptr(K_ref), _ptr(K_cur), Lcur, int(correct), int(bool(causal)),
+                                  float(scale), _ptr(stats), _ptr(top), _stream(Q.device)))
+    return stats, top
 
 
 def jensen_bias(Q: torch.Tensor, cache: KVCache, scale: float = 0.0) -> torch.Tensor:

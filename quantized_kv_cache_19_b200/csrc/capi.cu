@@ -7,6 +7,7 @@
 #include <string>
 
 #include "../../include/qkv.h"
+#include "fidelity.h"
 #include "qkv_internal.h"
 
 #define QKV_API extern "C" __attribute__((visibility("default")))
@@ -286,6 +287,53 @@ QKV_API qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, in
   p.wcoef = sc * sc / 24.0f;
   cudaError_t e = launch_jensen_bias(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "qkv_jensen_bias launch");
+  return QKV_OK;
+}
+
+QKV_API qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
+                                      const qkv_cache* cache, const void* K_ref, const void* K_cur,
+                                      int64_t L_cur, int32_t correct, int32_t causal_cur, float scale,
+                                      float* stats, int32_t* top, void* stream) {
+  t_last_error.clear();
+  qkv_status s = check_cache(cache);
+  if (s != QKV_OK) return s;
+  if (!in_dtype_ok(dtype)) return fail(QKV_ERR_UNSUPPORTED, "dtype must be F32 or BF16");
+  if (H_q < 1 || H_q % cache->H_kv)
+    return fail(QKV_ERR_INVALID_ARG, "H_q %d must be a positive multiple of H_kv %d", H_q,
+                cache->H_kv);
+  if (L_q < 0 || L_cur < 0) return fail(QKV_ERR_INVALID_ARG, "negative length");
+  if (correct < 0 || correct > 2) return fail(QKV_ERR_UNSUPPORTED, "correct must be 0, 1 or 2");
+  if (causal_cur != 0 && causal_cur != 1) return fail(QKV_ERR_INVALID_ARG, "causal_cur must be 0 or 1");
+  if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
+  if (cache->length + L_cur >= 2147483647LL)
+    return fail(QKV_ERR_UNSUPPORTED, "length + L_cur must be below 2^31 - 1");
+  if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
+  if (L_q == 0) return QKV_OK;
+  if (!Q || !stats) return fail(QKV_ERR_INVALID_ARG, "Q or stats is NULL");
+  if (cache->length > 0 && !K_ref) return fail(QKV_ERR_INVALID_ARG, "K_ref is NULL");
+  if (L_cur > 0 && !K_cur) return fail(QKV_ERR_INVALID_ARG, "K_cur is NULL");
+  if (!aligned16(Q) || !aligned16(stats) || (top && !aligned16(top)) ||
+      (cache->length > 0 && !aligned16(K_ref)) || (L_cur > 0 && !aligned16(K_cur)))
+    return fail(QKV_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const int64_t rows = static_cast<int64_t>(H_q / cache->H_kv) * L_q;
+  const int rpc = fidelity_rows_per_cta();
+  if ((rows + rpc - 1) / rpc > 2147483647LL || static_cast<int64_t>(cache->B) * cache->H_kv > 65535)
+    return fail(QKV_ERR_UNSUPPORTED, "grid too large");
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(cache->d));
+  FidelityParams p;
+  p.Q = Q; p.K_ref = K_ref; p.K_cur = K_cur;
+  p.k_codes = cache->k_codes; p.k_meta = cache->k_meta;
+  p.stats = stats; p.top = top;
+  p.Lq = L_q; p.Lc = cache->length; p.Lcur = L_cur; p.capacity = cache->capacity;
+  p.B = cache->B; p.Hq = H_q; p.Hkv = cache->H_kv; p.r = H_q / cache->H_kv;
+  p.bits = cache->bits; p.group = cache->group; p.n_groups = cache->d / cache->group;
+  p.correct = correct; p.causal = causal_cur;
+  p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
+  p.scale = sc;
+  p.wcoef = sc * sc / 24.0f;
+  p.ucoef = correct == 2 ? sc * sc * sc * sc / 2880.0f : 0.0f;
+  cudaError_t e = launch_attention_fidelity(p, cache->d, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention_fidelity launch");
   return QKV_OK;
 }
 

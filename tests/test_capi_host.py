@@ -96,3 +96,27 @@ def test_attention_rejections(lib):
     assert lib.corrected_attention_workspace_bytes(ctypes.byref(c2), 4, 16, 8, ctypes.byref(ws)) == 0
     assert lib.qkv_jensen_bias(q, api.QKV_BF16, 3, 16, ctypes.byref(c2), 0.0, P(0xC0000), None) == \
         api.QKV_ERR_INVALID_ARG
+
+
+def test_fidelity_rejections(lib):
+    c = _fake_cache(length=0)
+    P = ctypes.c_void_p
+    q, st = P(0x70000), P(0x80000)
+    call = lambda **kw: lib.attention_fidelity(
+        kw.get("Q", q), kw.get("dt", api.QKV_BF16), kw.get("Hq", 4), kw.get("Lq", 16), ctypes.byref(kw.get("c", c)),
+        kw.get("Kref", P(0xA0000)), kw.get("K", P(0xB0000)), kw.get("Lcur", 0), kw.get("corr", 1),
+        kw.get("causal", 0), kw.get("scale", 0.0), kw.get("stats", st), kw.get("top", None), None)
+    assert call() == api.QKV_ERR_INVALID_ARG                         # no keys at all
+    c2 = _fake_cache(length=100)
+    assert call(c=c2, Hq=3) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, dt=api.QKV_F16) == api.QKV_ERR_UNSUPPORTED
+    assert call(c=c2, corr=3) == api.QKV_ERR_UNSUPPORTED
+    assert call(c=c2, causal=2) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, Kref=None) == api.QKV_ERR_INVALID_ARG          # cached keys need K_ref
+    assert call(c=c2, Lcur=8, K=None) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, stats=None) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, top=P(0x90004)) == api.QKV_ERR_INVALID_ARG     # misaligned
+    assert call(c=c2, Kref=P(0xA0008)) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, scale=float("inf")) == api.QKV_ERR_INVALID_ARG
+    assert call(c=c2, Lcur=2 ** 31) == api.QKV_ERR_UNSUPPORTED       # key indices are int32
+    assert call(c=c2, Lq=0) == 0                                     # empty query chunk: no-op
