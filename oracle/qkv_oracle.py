@@ -26,6 +26,10 @@ Readings taken where the pages are silent (each one is also listed in the design
     operation a single correctly rounded fp32 operation, ties to even; a zero step gives code 0.
   * Packing: the codes of one (token, head) row form a little-endian bit string, channel c at
     bit c*bits, i.e. byte (c*bits)//8, bit (c*bits)%8.
+  * Per-channel keys (optional, key_block = T): every T consecutive cache positions (aligned to
+    position 0; the last block may be shorter) of one channel share a step and zero-point, by the
+    same fp32 arithmetic; codes are packed per token as above; values keep per-token groups.
+    The correction then uses each key's own per-channel steps.
   * Score scale: s = scale * q.k with scale = 1/sqrt(d) unless given; the correction is in the
     same scaled-score units. For a general scale the Taylor term is (scale^2/24) sum_c q_c^2
     Delta_c^2, which is the page's (1/(24 d)) sum_c q_c^2 Delta_{i,c}^2 at scale = 1/sqrt(d).
@@ -56,7 +60,7 @@ __all__ = [
     "META_DTYPES", "levels", "quantize", "pack_codes", "unpack_codes", "dequantize",
     "build_cache", "cache_rows", "log_sinhc", "jensen_bias_taylor", "jensen_bias_exact",
     "attention_rows", "corrected_attention", "merge_partials", "jensen_bias_taylor4",
-    "FIDELITY_TOPK", "fidelity_rows",
+    "FIDELITY_TOPK", "fidelity_rows", "quantize_tokens", "key_step_group",
 ]
 
 META_DTYPES = {"f32": np.float32, "f16": np.float16}
@@ -129,21 +133,82 @@ def dequantize(codes: np.ndarray, step: np.ndarray, zp: np.ndarray, group: int) 
     return xh.reshape(codes.shape)
 
 
-def build_cache(K: np.ndarray, V: np.ndarray, bits: int, group: int, meta: str = "f32") -> Dict:
-    """Quantise previous-chunk keys and values [B][Hkv][L][d] into the oracle's cache record."""
-    kc, ks, kz = quantize(K, bits, group, meta)
+def quantize_tokens(x: np.ndarray, bits: int, block: int, meta: str = "f32"
+                    ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Per-channel asymmetric min-max quantisation along the token axis (KIVI's key grouping, named
+    in [JB] 跨主題對比分析; [BLOG] groups along the sequence axis): tokens [k*block, (k+1)*block)
+    of one channel share one step and zero-point; the last block may be shorter.
+
+    x: [..., L, d]. Returns codes uint8 [..., L, d] (unpacked), step and zero-point
+    [..., ceil(L/block), d] in the meta dtype. The arithmetic of each (block, channel) is that of
+    `quantize` for one group: single fp32 IEEE operations in the same order.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    L, d = x.shape[-2], x.shape[-1]
+    nb = -(-L // block)
+    mt = META_DTYPES[meta]
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    step = np.zeros(x.shape[:-2] + (nb, d), dtype=mt)
+    zp = np.zeros(x.shape[:-2] + (nb, d), dtype=mt)
+    for k in range(nb):
+        xb = x[..., k * block:(k + 1) * block, :]
+        mn = xb.min(axis=-2)
+        mx = xb.max(axis=-2)
+        step32 = (mx - mn) / np.float32(levels(bits))
+        step[..., k, :] = step32.astype(mt)
+        zp[..., k, :] = mn.astype(mt)
+        stepf = step[..., k, :].astype(np.float32)
+        zpf = zp[..., k, :].astype(np.float32)
+        pos = stepf > 0
+        inv = np.zeros_like(stepf)
+        inv[pos] = np.float32(1.0) / stepf[pos]
+        t = (xb - zpf[..., None, :]) * inv[..., None, :]
+        code = np.clip(np.rint(t), 0, levels(bits))
+        codes[..., k * block:(k + 1) * block, :] = np.where(pos[..., None, :], code, 0).astype(np.uint8)
+    return codes, step, zp
+
+
+def build_cache(K: np.ndarray, V: np.ndarray, bits: int, group: int, meta: str = "f32",
+                key_block: int = 0) -> Dict:
+    """Quantise previous-chunk keys and values [B][Hkv][L][d] into the oracle's cache record.
+
+    key_block = 0: keys in groups of `group` channels per token, like values. key_block = T > 0: keys
+    per channel over blocks of T tokens (`quantize_tokens`); values stay per token.
+    """
+    if key_block:
+        kc, ks, kz = quantize_tokens(K, bits, key_block, meta)
+    else:
+        kc, ks, kz = quantize(K, bits, group, meta)
     vc, vs, vz = quantize(V, bits, group, meta)
-    return {"bits": bits, "group": group, "meta": meta,
+    return {"bits": bits, "group": group, "meta": meta, "key_block": key_block,
             "k_codes": kc, "k_step": ks, "k_zp": kz,
             "v_codes": vc, "v_step": vs, "v_zp": vz}
 
 
+def key_step_group(cache: Optional[Dict], d: int) -> int:
+    """Channels that share one key step within a key, as `cache_rows` returns the steps: `group` for
+    per-token key groups, 1 for per-channel keys."""
+    if cache is None:
+        return d
+    return 1 if cache.get("key_block") else cache["group"]
+
+
 def cache_rows(cache: Dict, b: int, h: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Dequantised keys, values [Lc][d] (fp64) and key steps [Lc][n_g] of one (batch, KV head)."""
+    """Dequantised keys, values [Lc][d] (fp64) and key steps of one (batch, KV head): [Lc][n_g] for
+    per-token key groups, [Lc][d] (each key's own per-channel steps) for per-channel keys."""
     g = cache["group"]
-    kh = dequantize(cache["k_codes"][b, h], cache["k_step"][b, h], cache["k_zp"][b, h], g)
+    T = cache.get("key_block", 0)
+    if T:
+        codes = cache["k_codes"][b, h]
+        Lc = codes.shape[0]
+        ks = np.repeat(cache["k_step"][b, h].astype(np.float64), T, axis=0)[:Lc]
+        kz = np.repeat(cache["k_zp"][b, h].astype(np.float64), T, axis=0)[:Lc]
+        kh = kz + ks * codes.astype(np.float64)
+    else:
+        kh = dequantize(cache["k_codes"][b, h], cache["k_step"][b, h], cache["k_zp"][b, h], g)
+        ks = cache["k_step"][b, h].astype(np.float64)
     vh = dequantize(cache["v_codes"][b, h], cache["v_step"][b, h], cache["v_zp"][b, h], g)
-    return kh, vh, cache["k_step"][b, h].astype(np.float64)
+    return kh, vh, ks
 
 
 # --------------------------------------------------------------------------------------------
@@ -270,7 +335,7 @@ def corrected_attention(Q: np.ndarray, cache: Optional[Dict], K_cur: np.ndarray,
     r = Hq // Hkv
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    group = cache["group"] if cache is not None else d
+    group = key_step_group(cache, d)
     if rows is None:
         O = np.zeros((B, Hq, Lq, d))
         LSE = np.zeros((B, Hq, Lq))
