@@ -309,6 +309,60 @@ def fidelity_leg(w, x, cache, dev, flush, steps: int = 10):
                       "top5_recall": round(st[..., 6].mean().item(), 5)}}
 
 
+def key_channel_leg(w, x, dev, flush, T: int = 32, steps: int = 10):
+    """Per-channel keys along tokens (blocks of T positions, KIVI's group size of 32) on the bench
+    workload: the whole-cache quantise-append (keys per channel, values per token; HBM-bound) and
+    corrected attention (correct=1) on the fp32 CUDA-core kernel that serves this layout, against
+    the fp32 FMA peak."""
+    props = torch.cuda.get_device_properties(dev)
+    sm_mhz = float(load_peaks()[0].get("sm_max_mhz", 1965.0))
+    fp32_peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+    hbm = float(load_peaks()[0]["hbm_gbs"])
+    cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc), w.meta, device=dev,
+                        key_block=T)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        ts = []
+        for i in range(steps + 3):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.mean(ts)
+
+    def quant():
+        cache.length = 0
+        api.kv_quantize_append(cache, x["K_src"], x["V_src"])
+
+    q_ms = timed(quant)
+    in_bytes = x["K_src"].element_size()
+    q_bytes = 2 * w.B * w.Hkv * w.Lc * w.d * in_bytes + cache.packed_bytes(w.Lc)
+    O = torch.empty_like(x["Q"])
+    LSE = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
+    a_ms = timed(lambda: api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1,
+                                                 causal=w.causal, out=O, lse=LSE))
+    if api.device_status() != 0:
+        raise RuntimeError("device status after the per-channel key leg")
+    flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
+    tf = flops / (a_ms * 1e-3) / 1e12
+    gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    del cache
+    return {"key_block": T,
+            "quantize_append_full_cache": {"bound": "hbm", "ms": round(q_ms, 4), "bytes": q_bytes,
+                                           "achieved_gbs": round(gbs, 1), "peak_gbs": hbm,
+                                           "frac": round(gbs / hbm, 4)},
+            "attention": {"kernel": "attention_f32_kernel (per-channel keys)", "bound": "alu",
+                          "ms_per_launch": round(a_ms, 4), "flops_per_launch": flops,
+                          "achieved": round(tf, 2), "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
+                          "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x max SM clock",
+                          "frac": round(tf / fp32_peak, 4)}}
+
+
 def run_ours(args, world, rank, local):
     w = WORKLOADS[args.workload]
     torch.cuda.set_device(local)
@@ -454,6 +508,8 @@ def run_ours(args, world, rank, local):
     }
     if not args.no_fidelity:
         result["fidelity"] = fidelity_leg(w, x, cache, dev, flush)
+    if not args.no_key_channel:
+        result["key_per_channel"] = key_channel_leg(w, x, dev, flush)
     if not args.no_decode:
         result["decode"] = decode_sweep(dev, peaks, flush)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -499,6 +555,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the few-query-rows (decode) sweep")
     ap.add_argument("--no-fidelity", action="store_true", help="skip the attention-fidelity diagnostics")
+    ap.add_argument("--no-key-channel", action="store_true", help="skip the per-channel key layout leg")
     ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
                     help="store the DRAM bytes per launch of an ncu report (taken on --workload) and exit")
     ap.add_argument("--record-command", default="", help="the command line that made the report")

@@ -32,7 +32,7 @@
 extern "C" {
 #endif
 
-#define QKV_ABI_VERSION 1
+#define QKV_ABI_VERSION 2
 /* Tokens per cache tile; a cache's capacity must be a multiple of it. */
 #define QKV_CACHE_TILE 128
 
@@ -64,6 +64,16 @@ typedef enum { QKV_F32 = 0, QKV_BF16 = 1, QKV_F16 = 2 } qkv_dtype;
  *  capacity         : tokens the buffers hold per (b, h); a positive multiple of QKV_CACHE_TILE.
  * Supported: d in {64, 128}; bits in {2, 4}; group in {32, 64, 128} dividing d;
  * meta_dtype in {QKV_F32, QKV_F16}.
+ *
+ * key_block = T in {32, 64, 128} selects per-channel keys along tokens instead (KIVI's key
+ * grouping, named in the summary's section 跨主題對比分析; the hotelren.com blog, section 3.1, groups
+ * along the sequence axis): the T cache positions [k T, (k+1) T) of one channel share one step and
+ * zero-point, computed over those tokens with the arithmetic above; codes are packed per token as
+ * above; values keep per-token groups.
+ *  k_meta (key_block = T) : meta_dtype [B][H_kv][capacity / T][d][2].
+ * Every append must then start at a multiple of T (an append may end inside a block; that block's
+ * meta comes from the tokens appended), and the correction uses each key's per-channel steps.
+ * key_block = 0 is the per-token layout; zero-initialise the field (and `reserved`).
  */
 typedef struct {
   int32_t B, H_kv, d, bits, group;
@@ -74,9 +84,18 @@ typedef struct {
   uint8_t* v_codes;
   void* k_meta;
   void* v_meta;
+  int32_t key_block;
+  int32_t reserved;
 } qkv_cache;
 
-/* Bytes of ONE codes buffer and of ONE meta buffer for the given cache shape (host only). */
+/*
+ * Bytes of each of the four buffers of the cache described by `shape` (its shape fields and
+ * key_block; pointers and length are ignored). Host only.
+ */
+qkv_status qkv_cache_layout_bytes(const qkv_cache* shape, size_t* k_codes_bytes, size_t* v_codes_bytes,
+                                  size_t* k_meta_bytes, size_t* v_meta_bytes);
+
+/* Bytes of ONE codes buffer and of ONE meta buffer for the per-token layout (host only). */
 qkv_status qkv_cache_bytes(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int32_t group,
                            int32_t meta_dtype, int64_t capacity, size_t* codes_bytes_each,
                            size_t* meta_bytes_each);
@@ -126,6 +145,8 @@ qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H
  *                 owned by the caller; NULL (or too small) runs the same attention without the
  *                 key split. Calls on one stream may reuse it; concurrent calls need their own.
  * L_cur = 0 and cache->length = 0 together are rejected (no keys at all).
+ * A cache with per-channel keys (key_block > 0) is served by an fp32 CUDA-core kernel for bf16 and
+ * fp32 inputs alike; it uses no workspace (corrected_attention_workspace_bytes() gives 0).
  */
 qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
                                const qkv_cache* cache, const void* K_cur, const void* V_cur,
@@ -156,7 +177,8 @@ qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int32_t H_q
 /*
  * The correction term alone, for checking: bias fp32 [B][H_q][L_q][cache->length] with
  * bias[b][hq][i][j] = (scale^2/24) * sum_c Q[b][hq][i][c]^2 * step_{j, c/group}^2, computed by
- * the same device functions corrected_attention uses (fp32).
+ * the same device functions corrected_attention uses (fp32). With per-channel keys (key_block > 0)
+ * step_{j,c} is the step of channel c in key j's block.
  */
 qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
                            const qkv_cache* cache, float scale, float* bias, void* stream);
@@ -181,7 +203,8 @@ qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, int64_t L_
  *           key j, length + t is current key t; -1 pads rows that see fewer than 5 keys. Recall
  *           counts the reference list's keys found in the quantised list, over min(5, keys seen).
  * Every score is fp32 (CUDA cores). Pointers are device pointers, 16-byte aligned, caller-owned;
- * nothing is allocated. length + L_cur must be below 2^31 - 1. Errors as corrected_attention.
+ * nothing is allocated. length + L_cur must be below 2^31 - 1; key_block must be 0 (else
+ * QKV_ERR_UNSUPPORTED). Errors as corrected_attention.
  */
 qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
                               const qkv_cache* cache, const void* K_ref, const void* K_cur,

@@ -32,7 +32,8 @@ class QkvCacheDesc(ctypes.Structure):
                 ("bits", ctypes.c_int32), ("group", ctypes.c_int32), ("meta_dtype", ctypes.c_int32),
                 ("capacity", ctypes.c_int64), ("length", ctypes.c_int64),
                 ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
-                ("k_meta", ctypes.c_void_p), ("v_meta", ctypes.c_void_p)]
+                ("k_meta", ctypes.c_void_p), ("v_meta", ctypes.c_void_p),
+                ("key_block", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class QkvError(RuntimeError):
@@ -49,6 +50,7 @@ _SIGS = {
     "qkv_last_error": (ctypes.c_char_p, []),
     "qkv_cache_bytes": (ctypes.c_int, [ctypes.c_int32] * 6 + [ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t),
                                                              ctypes.POINTER(ctypes.c_size_t)]),
+    "qkv_cache_layout_bytes": (ctypes.c_int, [ctypes.POINTER(QkvCacheDesc)] + [ctypes.POINTER(ctypes.c_size_t)] * 4),
     "kv_quantize_append": (ctypes.c_int, [ctypes.POINTER(QkvCacheDesc), _P, _P, ctypes.c_int32,
                                           ctypes.c_int64, _P]),
     "corrected_attention_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(QkvCacheDesc), ctypes.c_int32,
@@ -123,23 +125,29 @@ class KVCache:
     """Device buffers of a packed INT2/INT4 cache plus the C descriptor that points at them."""
 
     def __init__(self, B: int, H_kv: int, d: int, bits: int, group: int, capacity: int,
-                 meta: str = "f32", device="cuda"):
+                 meta: str = "f32", device="cuda", key_block: int = 0):
+        """key_block = T > 0: keys quantised per channel over blocks of T positions (values stay per
+        token in groups of `group` channels)."""
         lib = load_library()
         mcode, self.meta_torch = _META[meta]
-        cb, mb = ctypes.c_size_t(), ctypes.c_size_t()
-        _check(lib.qkv_cache_bytes(B, H_kv, d, bits, group, mcode, capacity, ctypes.byref(cb),
-                                   ctypes.byref(mb)))
+        shape = QkvCacheDesc(B, H_kv, d, bits, group, mcode, capacity, 0, None, None, None, None,
+                             key_block, 0)
+        kc, vc, km, vm = (ctypes.c_size_t() for _ in range(4))
+        _check(lib.qkv_cache_layout_bytes(ctypes.byref(shape), ctypes.byref(kc), ctypes.byref(vc),
+                                          ctypes.byref(km), ctypes.byref(vm)))
         self.device = torch.device(device)
         self.B, self.H_kv, self.d, self.bits, self.group, self.capacity, self.meta = \
             B, H_kv, d, bits, group, capacity, meta
+        self.key_block = key_block
         self.n_groups = d // group
-        self.k_codes = torch.zeros(cb.value, dtype=torch.uint8, device=self.device)
-        self.v_codes = torch.zeros(cb.value, dtype=torch.uint8, device=self.device)
-        self.k_meta = torch.zeros(mb.value // self.meta_torch.itemsize, dtype=self.meta_torch, device=self.device)
-        self.v_meta = torch.zeros_like(self.k_meta)
+        isz = self.meta_torch.itemsize
+        self.k_codes = torch.zeros(kc.value, dtype=torch.uint8, device=self.device)
+        self.v_codes = torch.zeros(vc.value, dtype=torch.uint8, device=self.device)
+        self.k_meta = torch.zeros(km.value // isz, dtype=self.meta_torch, device=self.device)
+        self.v_meta = torch.zeros(vm.value // isz, dtype=self.meta_torch, device=self.device)
         self.desc = QkvCacheDesc(B, H_kv, d, bits, group, mcode, capacity, 0,
                                  self.k_codes.data_ptr(), self.v_codes.data_ptr(),
-                                 self.k_meta.data_ptr(), self.v_meta.data_ptr())
+                                 self.k_meta.data_ptr(), self.v_meta.data_ptr(), key_block, 0)
 
     @property
     def length(self) -> int:
@@ -156,14 +164,21 @@ class KVCache:
         return t.view(self.B, self.H_kv, self.capacity, self.d * self.bits // 8)
 
     def meta_view(self, which: str) -> torch.Tensor:
+        """[B][H_kv][capacity][d/group][2]; per-channel keys: [B][H_kv][capacity/T][d][2]."""
+        if which == "k" and self.key_block:
+            return self.k_meta.view(self.B, self.H_kv, self.capacity // self.key_block, self.d, 2)
         t = self.k_meta if which == "k" else self.v_meta
         return t.view(self.B, self.H_kv, self.capacity, self.n_groups, 2)
 
     def packed_bytes(self, tokens: Optional[int] = None) -> int:
         """Bytes of codes + (step, zero-point) for `tokens` tokens of K and V."""
         n = self.length if tokens is None else tokens
-        per = self.d * self.bits // 8 + self.n_groups * 2 * self.meta_torch.itemsize
-        return 2 * self.B * self.H_kv * n * per
+        codes = self.d * self.bits // 8
+        v_meta = self.n_groups * 2 * self.meta_torch.itemsize
+        if self.key_block:
+            k_meta = -(-n // self.key_block) * self.d * 2 * self.meta_torch.itemsize
+            return self.B * self.H_kv * (n * (2 * codes + v_meta) + k_meta)
+        return 2 * self.B * self.H_kv * n * (codes + v_meta)
 
 
 def kv_quantize_append(cache: KVCache, K: torch.Tensor, V: torch.Tensor) -> None:

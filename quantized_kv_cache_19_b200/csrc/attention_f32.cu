@@ -9,6 +9,16 @@
 // One CTA of 128 threads per (128 packed query rows, batch * KV head); one thread per query row.
 // Keys are staged 32 at a time in shared memory as fp32 (cached keys dequantised with one fp32
 // FMA, zp + step * code), and every thread walks them in order.
+//
+// The same kernel serves caches whose keys are quantised per channel along tokens (KIVI's key
+// grouping, agents-report.net, section 跨主題對比分析; hotelren.com blog, section 3.1): every T
+// cache positions of a channel share one step. There the correction of [JB] 方法,
+// (scale^2 / 24) sum_c q_c^2 Delta_{j,c}^2, is the same for all keys of a block, so it is taken once
+// per row and 32-key tile (T is a multiple of 32) from the block's squared steps; inputs may be
+// bf16 or fp32 and O has the input type.
+#include <cuda_bf16.h>
+
+#include "channel.h"
 #include "qkv_common.cuh"
 #include "qkv_internal.h"
 #include "qkv_jensen.cuh"
@@ -24,13 +34,21 @@ __device__ __forceinline__ int code_at(const uint8_t* row, int c, int bits) {
   return (row[bit >> 3] >> (bit & 7)) & ((1 << bits) - 1);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p, int bits) {
+template <bool kF32In>
+__device__ __forceinline__ float ld_in(const void* base, int64_t i) {
+  if (kF32In) return static_cast<const float*>(base)[i];
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
+}
+
+// kChan: keys quantised per channel over blocks of T positions (meta [BH][capacity/T][D][2]);
+// otherwise per token in groups of p.group channels. kF32In: Q, K_cur, V_cur and O are fp32 (else bf16).
+template <int D, bool kChan, bool kF32In>
+__global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p, int bits, int T) {
   extern __shared__ float sm[];
   float* q_s = sm;                              // [128][D + 1]
   float* k_s = q_s + kRows * (D + 1);           // [kKT][D]
   float* v_s = k_s + kKT * D;                   // [kKT][D]
-  float* d2_s = v_s + kKT * D;                  // [kKT][4]
+  float* d2_s = v_s + kKT * D;                  // [kKT][4]; per-channel keys: [D] squared steps
   const int t = threadIdx.x;
   const int m_tile = blockIdx.x;
   const int bh = blockIdx.y;
@@ -47,12 +65,13 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
   const int G = p.group, NG = p.n_groups;
   const int row_codes = D * bits / 8;
 
+  const float ucoef = p.ucoef_log2 * 0.69314718055994530942f;
   float w[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
   float u[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
-  const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * 4;
+  const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * (kF32In ? 4 : 2);
   if (valid_row) {
-    if (p.correct) query_group_powers<D>(qrow, true, G, wcoef, p.ucoef_log2 * 0.69314718055994530942f, w, u);
-    for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = reinterpret_cast<const float*>(qrow)[c];
+    if (!kChan && p.correct) query_group_powers<D>(qrow, kF32In, G, wcoef, ucoef, w, u);
+    for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = ld_in<kF32In>(qrow, c);
   } else {
     for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = 0.f;
   }
@@ -72,29 +91,47 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
       if (key < p.Lc) {
         const int64_t row = static_cast<int64_t>(bh) * p.capacity + key;
         const int g = c / G;
+        // key meta: per (token, group), or per (block of T tokens, channel)
+        const int64_t kmi = kChan ? ((static_cast<int64_t>(bh) * (p.capacity / T) + key / T) * D + c) * 2
+                                  : (row * NG + g) * 2;
         float ks, kz, vs, vz;
         if (p.meta_f16) {
-          const __half* km = static_cast<const __half*>(p.k_meta) + (row * NG + g) * 2;
+          const __half* km = static_cast<const __half*>(p.k_meta) + kmi;
           const __half* vm = static_cast<const __half*>(p.v_meta) + (row * NG + g) * 2;
           ks = __half2float(km[0]); kz = __half2float(km[1]);
           vs = __half2float(vm[0]); vz = __half2float(vm[1]);
         } else {
-          const float* km = static_cast<const float*>(p.k_meta) + (row * NG + g) * 2;
+          const float* km = static_cast<const float*>(p.k_meta) + kmi;
           const float* vm = static_cast<const float*>(p.v_meta) + (row * NG + g) * 2;
           ks = km[0]; kz = km[1]; vs = vm[0]; vz = vm[1];
         }
         kv = fmaf(ks, static_cast<float>(code_at(p.k_codes + row * row_codes, c, bits)), kz);
         vv = fmaf(vs, static_cast<float>(code_at(p.v_codes + row * row_codes, c, bits)), vz);
-        if (c % G == 0) d2_s[kk * 4 + g] = ks * ks;
+        if (kChan) {
+          if (kk == 0) d2_s[c] = ks * ks;        // the tile lies in one key block (T % 32 == 0)
+        } else if (c % G == 0) {
+          d2_s[kk * 4 + g] = ks * ks;
+        }
       } else if (key < total) {
         const int64_t row = static_cast<int64_t>(bh) * p.Lcur + (key - p.Lc);
-        kv = static_cast<const float*>(p.K_cur)[row * D + c];
-        vv = static_cast<const float*>(p.V_cur)[row * D + c];
+        kv = ld_in<kF32In>(p.K_cur, row * D + c);
+        vv = ld_in<kF32In>(p.V_cur, row * D + c);
       }
       k_s[kk * D + c] = kv;
       v_s[kk * D + c] = vv;
     }
     __syncthreads();
+    // Per-channel keys: the tile's correction for this row, sum_c w_c Delta_c^2 (minus the fourth-
+    // order term sum_c u_c Delta_c^4 when correct = 2), one pass over the block's squared steps.
+    float tile_b = 0.f;
+    if (kChan && p.correct && k0 < p.Lc) {
+      for (int c = 0; c < D; ++c) {
+        const float q2 = q_s[t * (D + 1) + c] * q_s[t * (D + 1) + c];
+        const float d2 = d2_s[c];
+        tile_b = fmaf(wcoef * q2, d2, tile_b);
+        if (p.correct == 2) tile_b = fmaf(-ucoef * (q2 * q2), d2 * d2, tile_b);
+      }
+    }
     for (int kk = 0; kk < kKT; ++kk) {
       const int64_t key = k0 + kk;
       if (key >= total) break;
@@ -103,7 +140,9 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
       float s = 0.f;
       for (int c = 0; c < D; ++c) s = fmaf(q_s[t * (D + 1) + c], k_s[kk * D + c], s);
       s *= scale;
-      if (cached && p.correct) {
+      if (kChan) {
+        if (cached) s -= tile_b;
+      } else if (cached && p.correct) {
         float d2[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
         for (int g = 0; g < NG; ++g) d2[g] = d2_s[kk * 4 + g];
         s -= jensen_term(w, d2, NG);
@@ -125,10 +164,16 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
     }
   }
   if (valid_row) {
-    float* orow = static_cast<float*>(p.O) + out_row * D;
     const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (kF32In) {
+      float* orow = static_cast<float*>(p.O) + out_row * D;
 #pragma unroll
-    for (int c = 0; c < D; ++c) orow[c] = o[c] * inv;
+      for (int c = 0; c < D; ++c) orow[c] = o[c] * inv;
+    } else {
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.O) + out_row * D;
+#pragma unroll
+      for (int c = 0; c < D; ++c) orow[c] = __float2bfloat16_rn(o[c] * inv);
+    }
     p.LSE[out_row] = l > 0.f ? m + logf(l) : -INFINITY;
   }
 }
@@ -157,23 +202,65 @@ __global__ void __launch_bounds__(256) jensen_bias_kernel(const BiasParams p) {
   p.bias[qrow * p.Lc + j] = jensen_term(w, d2, p.n_groups);
 }
 
-template <int D>
-cudaError_t launch_f32(const AttnParams& p, int bits, cudaStream_t stream) {
-  const size_t smem = (kRows * (D + 1) + 2 * kKT * D + kKT * 4) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(attention_f32_kernel<D>,
+// Correction term alone for per-channel keys: b = (scale^2 / 24) sum_c q_c^2 Delta_{block(j), c}^2.
+template <int D, bool kF32In>
+__global__ void __launch_bounds__(256) jensen_bias_channel_kernel(const BiasParams p, int T) {
+  const int64_t qrow = blockIdx.x;
+  const int64_t j = static_cast<int64_t>(blockIdx.y) * blockDim.x + threadIdx.x;
+  if (j >= p.Lc) return;
+  const int64_t bhq = qrow / p.Lq;
+  const int64_t b = bhq / p.Hq, hq = bhq % p.Hq;
+  const int64_t hkv = hq / p.r;
+  const int64_t blk = (b * p.Hkv + hkv) * (p.capacity / T) + j / T;
+  float acc = 0.f;
+  for (int c = 0; c < D; ++c) {
+    const float q = ld_in<kF32In>(p.Q, qrow * D + c);
+    const float s = p.meta_f16 ? __half2float(static_cast<const __half*>(p.k_meta)[(blk * D + c) * 2])
+                               : static_cast<const float*>(p.k_meta)[(blk * D + c) * 2];
+    acc = fmaf(p.wcoef * (q * q), s * s, acc);
+  }
+  p.bias[qrow * p.Lc + j] = acc;
+}
+
+template <int D, bool kChan, bool kF32In>
+cudaError_t launch_f32(const AttnParams& p, int bits, int T, cudaStream_t stream) {
+  const size_t smem = (kRows * (D + 1) + 2 * kKT * D + (kChan ? D : kKT * 4)) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(attention_f32_kernel<D, kChan, kF32In>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(p.r) * p.Lq;
   dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), static_cast<unsigned>(p.B * p.Hkv));
-  attention_f32_kernel<D><<<grid, kRows, smem, stream>>>(p, bits);
+  attention_f32_kernel<D, kChan, kF32In><<<grid, kRows, smem, stream>>>(p, bits, T);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attention_f32(const AttnParams& p, int d, int bits, cudaStream_t stream) {
-  return d == 128 ? launch_f32<128>(p, bits, stream) : launch_f32<64>(p, bits, stream);
+  return d == 128 ? launch_f32<128, false, true>(p, bits, 0, stream)
+                  : launch_f32<64, false, true>(p, bits, 0, stream);
+}
+
+cudaError_t launch_attention_channel(const AttnParams& p, int d, int bits, int T, cudaStream_t stream) {
+  if (p.in_f32) {
+    return d == 128 ? launch_f32<128, true, true>(p, bits, T, stream)
+                    : launch_f32<64, true, true>(p, bits, T, stream);
+  }
+  return d == 128 ? launch_f32<128, true, false>(p, bits, T, stream)
+                  : launch_f32<64, true, false>(p, bits, T, stream);
+}
+
+cudaError_t launch_jensen_bias_channel(const BiasParams& p, int T, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(p.B * p.Hq * p.Lq), static_cast<unsigned>((p.Lc + 255) / 256));
+  if (p.d == 128) {
+    if (p.in_f32) jensen_bias_channel_kernel<128, true><<<grid, 256, 0, stream>>>(p, T);
+    else jensen_bias_channel_kernel<128, false><<<grid, 256, 0, stream>>>(p, T);
+  } else {
+    if (p.in_f32) jensen_bias_channel_kernel<64, true><<<grid, 256, 0, stream>>>(p, T);
+    else jensen_bias_channel_kernel<64, false><<<grid, 256, 0, stream>>>(p, T);
+  }
+  return cudaGetLastError();
 }
 
 cudaError_t launch_jensen_bias(const BiasParams& p, cudaStream_t stream) {

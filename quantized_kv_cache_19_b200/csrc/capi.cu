@@ -7,6 +7,7 @@
 #include <string>
 
 #include "../../include/qkv.h"
+#include "channel.h"
 #include "fidelity.h"
 #include "qkv_internal.h"
 
@@ -68,6 +69,12 @@ qkv_status check_shape(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int32_t
   return QKV_OK;
 }
 
+qkv_status check_key_block(int32_t key_block) {
+  if (key_block != 0 && key_block != 32 && key_block != 64 && key_block != 128)
+    return fail(QKV_ERR_UNSUPPORTED, "key_block %d not supported (0, 32, 64, 128)", key_block);
+  return QKV_OK;
+}
+
 qkv_status check_cache(const qkv_cache* c) {
   if (c == nullptr) return fail(QKV_ERR_INVALID_ARG, "cache is NULL");
   qkv_status s = check_shape(c->B, c->H_kv, c->d, c->bits, c->group, c->meta_dtype, c->capacity);
@@ -80,7 +87,7 @@ qkv_status check_cache(const qkv_cache* c) {
   if (!aligned16(c->k_codes) || !aligned16(c->v_codes) || !aligned16(c->k_meta) ||
       !aligned16(c->v_meta))
     return fail(QKV_ERR_INVALID_ARG, "cache buffers must be 16-byte aligned");
-  return QKV_OK;
+  return check_key_block(c->key_block);
 }
 
 bool in_dtype_ok(int32_t dt) { return dt == QKV_F32 || dt == QKV_BF16; }
@@ -119,6 +126,23 @@ QKV_API qkv_status qkv_cache_bytes(int32_t B, int32_t H_kv, int32_t d, int32_t b
   return QKV_OK;
 }
 
+QKV_API qkv_status qkv_cache_layout_bytes(const qkv_cache* c, size_t* k_codes, size_t* v_codes,
+                                          size_t* k_meta, size_t* v_meta) {
+  t_last_error.clear();
+  if (c == nullptr) return fail(QKV_ERR_INVALID_ARG, "cache is NULL");
+  qkv_status s = check_shape(c->B, c->H_kv, c->d, c->bits, c->group, c->meta_dtype, c->capacity);
+  if (s != QKV_OK) return s;
+  s = check_key_block(c->key_block);
+  if (s != QKV_OK) return s;
+  if (!k_codes || !v_codes || !k_meta || !v_meta) return fail(QKV_ERR_INVALID_ARG, "NULL output");
+  const size_t tokens = static_cast<size_t>(c->B) * c->H_kv * static_cast<size_t>(c->capacity);
+  const size_t mb = c->meta_dtype == QKV_F16 ? 2 : 4;
+  *k_codes = *v_codes = tokens * (c->d * c->bits / 8);
+  *v_meta = tokens * (c->d / c->group) * 2 * mb;
+  *k_meta = c->key_block ? tokens / c->key_block * c->d * 2 * mb : *v_meta;
+  return QKV_OK;
+}
+
 QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const void* V,
                                       int32_t in_dtype, int64_t L_new, void* stream) {
   t_last_error.clear();
@@ -143,8 +167,25 @@ QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const voi
   p.start = cache->length;
   p.d = cache->d;
   p.group = cache->group;
-  cudaError_t e = launch_quantize_append(p, in_dtype, cache->meta_dtype, cache->bits,
-                                         static_cast<cudaStream_t>(stream));
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cache->key_block) {
+    // Keys per channel over blocks of key_block positions: an append starts a new block.
+    if (cache->length % cache->key_block)
+      return fail(QKV_ERR_UNSUPPORTED,
+                  "per-channel key blocks: the cache length %lld is not a multiple of key_block %d "
+                  "(only the last append may end inside a block)",
+                  static_cast<long long>(cache->length), cache->key_block);
+    ChanQuantParams kp;
+    kp.K = K; kp.k_codes = cache->k_codes; kp.k_meta = cache->k_meta;
+    kp.BH = p.BH; kp.L_new = L_new; kp.capacity = cache->capacity; kp.start = cache->length;
+    kp.d = cache->d; kp.T = cache->key_block;
+    if (kp.BH > 65535 || (L_new + kp.T - 1) / kp.T > 2147483647LL)
+      return fail(QKV_ERR_UNSUPPORTED, "grid too large");
+    p.K = nullptr;                    // the per-token kernel quantises V only
+    cudaError_t e = launch_quantize_keys_channel(kp, in_dtype, cache->meta_dtype, cache->bits, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_quantize_append (keys) launch");
+  }
+  cudaError_t e = launch_quantize_append(p, in_dtype, cache->meta_dtype, cache->bits, st);
   if (e != cudaSuccess) return cuda_fail(e, "kv_quantize_append launch");
   cache->length += L_new;
   return QKV_OK;
@@ -186,7 +227,7 @@ QKV_API qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, i
   if (!bytes) return fail(QKV_ERR_INVALID_ARG, "NULL output");
   if (H_q < 1 || H_q % cache->H_kv || L_q < 0 || L_cur < 0)
     return fail(QKV_ERR_INVALID_ARG, "bad H_q / L_q / L_cur");
-  *bytes = split_workspace_bytes(cache, H_q, L_q, attention_splits(cache, H_q, L_q));
+  *bytes = cache->key_block ? 0 : split_workspace_bytes(cache, H_q, L_q, attention_splits(cache, H_q, L_q));
   return QKV_OK;
 }
 
@@ -239,6 +280,11 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   p.ws_o = nullptr;
   p.ws_lse = nullptr;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cache->key_block) {
+    e = launch_attention_channel(p, cache->d, cache->bits, cache->key_block, st);
+    if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");
+    return QKV_OK;
+  }
   if (dtype == QKV_F32) {
     e = launch_attention_f32(p, cache->d, cache->bits, st);
     if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");
@@ -285,7 +331,9 @@ QKV_API qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, in
   p.d = cache->d; p.group = cache->group; p.n_groups = cache->d / cache->group;
   p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
   p.wcoef = sc * sc / 24.0f;
-  cudaError_t e = launch_jensen_bias(p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = cache->key_block
+                      ? launch_jensen_bias_channel(p, cache->key_block, static_cast<cudaStream_t>(stream))
+                      : launch_jensen_bias(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "qkv_jensen_bias launch");
   return QKV_OK;
 }
@@ -307,6 +355,8 @@ QKV_API qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q,
   if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
   if (cache->length + L_cur >= 2147483647LL)
     return fail(QKV_ERR_UNSUPPORTED, "length + L_cur must be below 2^31 - 1");
+  if (cache->key_block)
+    return fail(QKV_ERR_UNSUPPORTED, "attention_fidelity: per-channel key blocks are not supported");
   if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
   if (L_q == 0) return QKV_OK;
   if (!Q || !stats) return fail(QKV_ERR_INVALID_ARG, "Q or stats is NULL");
@@ -416,7 +466,7 @@ QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int
   if ((rows + 127) / 128 > 2147483647LL || static_cast<int64_t>(cache->B) * cache->H_kv > 65535)
     return fail(QKV_ERR_UNSUPPORTED, "grid too large");
   // The key split this shape takes, and whether its scratch fits the library's array.
-  const int n = dtype == QKV_BF16 ? attention_splits(cache, H_q, L_q) : 1;
+  const int n = dtype == QKV_BF16 && !cache->key_block ? attention_splits(cache, H_q, L_q) : 1;
   const size_t need = split_workspace_bytes(cache, H_q, L_q, n);
   if (need > kNoAllocScratchBytes)
     return fail(QKV_ERR_UNSUPPORTED,
@@ -452,8 +502,9 @@ QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int
   p.ws_o = scratch;
   p.ws_lse = scratch ? scratch + static_cast<size_t>(n) * p.rows_all * cache->d : nullptr;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  e = dtype == QKV_F32 ? launch_attention_f32(p, cache->d, cache->bits, st)
-                       : launch_attention_bf16(p, cache->d, cache->bits, st);
+  e = cache->key_block ? launch_attention_channel(p, cache->d, cache->bits, cache->key_block, st)
+      : dtype == QKV_F32 ? launch_attention_f32(p, cache->d, cache->bits, st)
+                         : launch_attention_bf16(p, cache->d, cache->bits, st);
   if (e != cudaSuccess) return cuda_fail(e, "corrected_attention_noalloc launch");
   if (n > 1) {
     e = launch_split_merge(p.ws_o, p.ws_lse, n, p.rows_all, cache->d, O, LSE, st);

@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
   constexpr int kPasses = 4;
   constexpr int kRowsPerBlock = kRowsPerPass * kPasses;
   const int tensor = blockIdx.z;
+  if (tensor == 0 && p.K == nullptr) return;  // keys quantised per channel by another kernel
   const int lr = threadIdx.x % kTpr;          // lane within the row: channels 8*lr .. 8*lr+7
   const int pr = threadIdx.x / kTpr;          // row within the pass
   const InT* src_base = static_cast<const InT*>(tensor ? p.V : p.K);

@@ -14,7 +14,7 @@ def test_exports_every_header_function(lib):
             "qkv_last_error", "qkv_abi_version"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.qkv_abi_version() == 1
+    assert lib.qkv_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -120,3 +120,47 @@ def test_fidelity_rejections(lib):
     assert call(c=c2, scale=float("inf")) == api.QKV_ERR_INVALID_ARG
     assert call(c=c2, Lcur=2 ** 31) == api.QKV_ERR_UNSUPPORTED       # key indices are int32
     assert call(c=c2, Lq=0) == 0                                     # empty query chunk: no-op
+
+
+def test_descriptor_size_matches_the_header():
+    # 6 int32, 2 int64, 4 pointers, key_block and reserved
+    assert ctypes.sizeof(api.QkvCacheDesc) == 6 * 4 + 2 * 8 + 4 * 8 + 2 * 4
+
+
+@pytest.mark.parametrize("key_block,meta,k_meta", [
+    (0, api.QKV_F32, 2 * 256 * 2 * 2 * 4),            # per-token: [B][H][cap][d/group][2]
+    (32, api.QKV_F32, 2 * (256 // 32) * 128 * 2 * 4),  # per-channel: [B][H][cap/T][d][2]
+    (128, api.QKV_F16, 2 * (256 // 128) * 128 * 2 * 2),
+])
+def test_layout_bytes(lib, key_block, meta, k_meta):
+    c = _fake_cache(key_block=key_block, meta_dtype=meta)
+    out = [ctypes.c_size_t() for _ in range(4)]
+    assert lib.qkv_cache_layout_bytes(ctypes.byref(c), *[ctypes.byref(o) for o in out]) == 0
+    kc, vc, km, vm = (o.value for o in out)
+    msz = 4 if meta == api.QKV_F32 else 2
+    assert kc == vc == 2 * 256 * 32
+    assert vm == 2 * 256 * 2 * 2 * msz
+    assert km == k_meta
+
+
+def test_key_block_rejections(lib):
+    P = ctypes.c_void_p
+    out = [ctypes.c_size_t() for _ in range(4)]
+    bad = _fake_cache(key_block=16)
+    assert lib.qkv_cache_layout_bytes(ctypes.byref(bad), *[ctypes.byref(o) for o in out]) == \
+        api.QKV_ERR_UNSUPPORTED
+    assert lib.kv_quantize_append(ctypes.byref(bad), P(0x50000), P(0x60000), api.QKV_BF16, 8, None) == \
+        api.QKV_ERR_UNSUPPORTED
+    # appends must start on a block boundary; the cache is left unchanged
+    c = _fake_cache(key_block=32, length=40)
+    assert lib.kv_quantize_append(ctypes.byref(c), P(0x50000), P(0x60000), api.QKV_BF16, 8, None) == \
+        api.QKV_ERR_UNSUPPORTED
+    assert c.length == 40 and b"key_block" in lib.qkv_last_error()
+    # no key split and no workspace for per-channel keys
+    c2 = _fake_cache(key_block=64, length=256, capacity=256)
+    ws = ctypes.c_size_t(1)
+    assert lib.corrected_attention_workspace_bytes(ctypes.byref(c2), 2, 1, 1, ctypes.byref(ws)) == 0
+    assert ws.value == 0
+    st = P(0x80000)
+    assert lib.attention_fidelity(P(0x70000), api.QKV_BF16, 2, 4, ctypes.byref(c2), P(0xA0000), None, 0,
+                                  1, 0, 0.0, st, None, None) == api.QKV_ERR_UNSUPPORTED
