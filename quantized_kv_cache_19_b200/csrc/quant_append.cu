@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
   constexpr int kRowsPerPass = 256 / kTpr;
   constexpr int kPasses = 4;
   constexpr int kRowsPerBlock = kRowsPerPass * kPasses;
+  static_assert(kTpg >= kPasses, "each row's step is computed by its own lane of the group");
   const int tensor = blockIdx.z;
   if (tensor == 0 && p.K == nullptr) return;  // keys quantised per channel by another kernel
   const int lr = threadIdx.x % kTpr;          // lane within the row: channels 8*lr .. 8*lr+7
@@ -136,26 +137,47 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
         for (int k = 0; k < 8; ++k) x[u][k] = 0.f;
       }
     }
+    // Group min/max of every row, reduced over the group's lanes (all of them get the result).
+    float mn[kPasses], mx[kPasses];
 #pragma unroll
     for (int u = 0; u < kPasses; ++u) {
-      const int64_t t = t0 + u * kRowsPerPass;
-      float mn = fmin3(fmin3(x[u][0], x[u][1], x[u][2]), fmin3(x[u][3], x[u][4], x[u][5]), fminf(x[u][6], x[u][7]));
-      float mx = fmax3(fmax3(x[u][0], x[u][1], x[u][2]), fmax3(x[u][3], x[u][4], x[u][5]), fmaxf(x[u][6], x[u][7]));
+      mn[u] = fmin3(fmin3(x[u][0], x[u][1], x[u][2]), fmin3(x[u][3], x[u][4], x[u][5]), fminf(x[u][6], x[u][7]));
+      mx[u] = fmax3(fmax3(x[u][0], x[u][1], x[u][2]), fmax3(x[u][3], x[u][4], x[u][5]), fmaxf(x[u][6], x[u][7]));
 #pragma unroll
       for (int off = 1; off < kTpg; off <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mn[u] = fminf(mn[u], __shfl_xor_sync(0xffffffffu, mn[u], off));
+        mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xffffffffu, mx[u], off));
       }
+    }
+    // Step, zero-point and reciprocal of a group: lane j of the group (kTpg >= kPasses lanes)
+    // computes them for row j % kPasses only, writes that row's meta, and the group's lanes read
+    // them back with shuffles. The arithmetic is the same single IEEE operations for every row.
+    const int jg = lr % kTpg;                    // lane within the group
+    const int uo = jg % kPasses;                 // the row this lane takes
+    float mn_o = mn[0], mx_o = mx[0];
+#pragma unroll
+    for (int u = 1; u < kPasses; ++u)
+      if (uo == u) { mn_o = mn[u]; mx_o = mx[u]; }
+    const float step32 = __fdiv_rn(__fsub_rn(mx_o, mn_o), static_cast<float>(kLevels));
+    const MetaT step_m = MetaOps<MetaT>::store(step32);
+    const MetaT zp_m = MetaOps<MetaT>::store(mn_o);
+    const float step_o = MetaOps<MetaT>::load(step_m);
+    const float zp_o = MetaOps<MetaT>::load(zp_m);
+    const float inv_o = step_o > 0.f ? __frcp_rn(step_o) : 0.f;
+    {
+      const int64_t t = t0 + uo * kRowsPerPass;
+      if (jg < kPasses && t < p.L_new) {
+        const int64_t dst_row = bh * p.capacity + p.start + t;
+        MetaOps<MetaT>::put_pair(meta_base + (dst_row * kNG + lr / kTpg) * 2, step_m, zp_m);
+      }
+    }
+    const int lane0 = (threadIdx.x & 31) - jg;  // first lane of this group in the warp
+#pragma unroll
+    for (int u = 0; u < kPasses; ++u) {
+      const float zp = __shfl_sync(0xffffffffu, zp_o, lane0 + u);
+      const float inv = __shfl_sync(0xffffffffu, inv_o, lane0 + u);
+      const int64_t t = t0 + u * kRowsPerPass;
       if (t >= p.L_new) continue;
-
-      const float step32 = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(kLevels));
-      const MetaT step_m = MetaOps<MetaT>::store(step32);
-      const MetaT zp_m = MetaOps<MetaT>::store(mn);
-      const float step = MetaOps<MetaT>::load(step_m);
-      const float zp = MetaOps<MetaT>::load(zp_m);
-      const bool pos = step > 0.f;
-      const float inv = pos ? __frcp_rn(step) : 0.f;
-
       const uint32_t packed = pack_codes8<BITS, !std::is_same<MetaT, float>::value>(x[u], zp, inv);
       const int64_t dst_row = bh * p.capacity + p.start + t;
       uint8_t* codes = codes_base + dst_row * (D * BITS / 8) + lr * BITS;
@@ -164,7 +186,6 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
       } else {
         *reinterpret_cast<uint32_t*>(codes) = packed;
       }
-      if ((lr % kTpg) == 0) MetaOps<MetaT>::put_pair(meta_base + (dst_row * kNG + lr / kTpg) * 2, step_m, zp_m);
     }
   }
 }
