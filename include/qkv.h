@@ -203,8 +203,8 @@ qkv_status qkv_jensen_bias(const void* Q, int32_t dtype, int32_t H_q, int64_t L_
  *           key j, length + t is current key t; -1 pads rows that see fewer than 5 keys. Recall
  *           counts the reference list's keys found in the quantised list, over min(5, keys seen).
  * Every score is fp32 (CUDA cores). Pointers are device pointers, 16-byte aligned, caller-owned;
- * nothing is allocated. length + L_cur must be below 2^31 - 1; key_block must be 0 (else
- * QKV_ERR_UNSUPPORTED). Errors as corrected_attention.
+ * nothing is allocated. length + L_cur must be below 2^31 - 1. Caches with per-channel keys
+ * (key_block > 0) are supported. Errors as corrected_attention.
  */
 qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
                               const qkv_cache* cache, const void* K_ref, const void* K_cur,

@@ -81,8 +81,17 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
   float m = -INFINITY, l = 0.f;
   const int64_t lim_cur = p.causal ? qi + (p.Lcur - p.Lq) + 1 : p.Lcur;   // current keys this row sees
 
-  const int64_t total = p.Lc + p.Lcur;
-  for (int64_t k0 = 0; k0 < total; k0 += kKT) {
+  // Keys [k_begin, total) of this CTA. With a split over the cached keys (n_split > 1, grid z),
+  // split z takes the 32-key cached tiles [z T / n, (z+1) T / n) and the last split also the
+  // current chunk; the partial O (normalised) and LSE go to the workspace for the merge.
+  int64_t k_begin = 0, total = p.Lc + p.Lcur;
+  if (p.n_split > 1) {
+    const int64_t tiles = (p.Lc + kKT - 1) / kKT;
+    const int z = blockIdx.z;
+    k_begin = tiles * z / p.n_split * kKT;
+    if (z + 1 < p.n_split) total = tiles * (z + 1) / p.n_split * kKT;
+  }
+  for (int64_t k0 = k_begin; k0 < total; k0 += kKT) {
     __syncthreads();
     for (int e = t; e < kKT * D; e += kRows) {
       const int kk = e / D, c = e % D;
@@ -163,7 +172,14 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
       for (int c = 0; c < D; ++c) o[c] = fmaf(pk, v_s[kk * D + c], o[c]);
     }
   }
-  if (valid_row) {
+  if (valid_row && p.n_split > 1) {
+    const int64_t prow = static_cast<int64_t>(blockIdx.z) * p.rows_all + out_row;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* orow = p.ws_o + prow * D;
+#pragma unroll
+    for (int c = 0; c < D; ++c) orow[c] = o[c] * inv;
+    p.ws_lse[prow] = l > 0.f ? m + logf(l) : -INFINITY;
+  } else if (valid_row) {
     const float inv = l > 0.f ? 1.f / l : 0.f;
     if (kF32In) {
       float* orow = static_cast<float*>(p.O) + out_row * D;
@@ -230,7 +246,8 @@ cudaError_t launch_f32(const AttnParams& p, int bits, int T, cudaStream_t stream
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int64_t rows = static_cast<int64_t>(p.r) * p.Lq;
-  dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), static_cast<unsigned>(p.B * p.Hkv));
+  dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), static_cast<unsigned>(p.B * p.Hkv),
+            static_cast<unsigned>(p.n_split > 1 ? p.n_split : 1));
   attention_f32_kernel<D, kChan, kF32In><<<grid, kRows, smem, stream>>>(p, bits, T);
   return cudaGetLastError();
 }
@@ -241,6 +258,9 @@ cudaError_t launch_attention_f32(const AttnParams& p, int d, int bits, cudaStrea
   return d == 128 ? launch_f32<128, false, true>(p, bits, 0, stream)
                   : launch_f32<64, false, true>(p, bits, 0, stream);
 }
+
+int channel_rows_per_cta() { return kRows; }
+int channel_tile_keys() { return kKT; }
 
 cudaError_t launch_attention_channel(const AttnParams& p, int d, int bits, int T, cudaStream_t stream) {
   if (p.in_f32) {

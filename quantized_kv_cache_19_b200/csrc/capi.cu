@@ -213,6 +213,29 @@ static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
   return n < 1 ? 1 : static_cast<int>(n);
 }
 
+// Splits of the cached keys for the per-channel-key kernel (bf16 inputs): as for the tensor-core
+// kernel, only when the (row tile, batch * KV head) grid would leave more than half of the SMs idle
+// (few query rows per KV head). Splitting fuller grids was measured slower: this CUDA-core kernel
+// gains nothing from a second CTA on an SM. 1 = no split.
+static int channel_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
+  if (L_q <= 0 || c->length <= 0) return 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  const int64_t rows = static_cast<int64_t>(H_q / c->H_kv) * L_q;
+  const int64_t rpc = channel_rows_per_cta();
+  const int64_t ctas = (rows + rpc - 1) / rpc * c->B * c->H_kv;
+  const int64_t tiles = (c->length + channel_tile_keys() - 1) / channel_tile_keys();
+  if (ctas * 2 > sms || tiles < 2) return 1;
+  int64_t n = sms / ctas;
+  if (n > tiles) n = tiles;
+  if (n > 32) n = 32;
+  return n < 1 ? 1 : static_cast<int>(n);
+}
+
 static size_t split_workspace_bytes(const qkv_cache* c, int32_t H_q, int64_t L_q, int n) {
   if (n <= 1) return 0;
   const size_t rows_all = static_cast<size_t>(c->B) * H_q * L_q;
@@ -227,7 +250,9 @@ QKV_API qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, i
   if (!bytes) return fail(QKV_ERR_INVALID_ARG, "NULL output");
   if (H_q < 1 || H_q % cache->H_kv || L_q < 0 || L_cur < 0)
     return fail(QKV_ERR_INVALID_ARG, "bad H_q / L_q / L_cur");
-  *bytes = cache->key_block ? 0 : split_workspace_bytes(cache, H_q, L_q, attention_splits(cache, H_q, L_q));
+  // The per-channel-key kernel splits only bf16 inputs; this size covers them (fp32 inputs ignore it).
+  const int n = cache->key_block ? channel_splits(cache, H_q, L_q) : attention_splits(cache, H_q, L_q);
+  *bytes = split_workspace_bytes(cache, H_q, L_q, n);
   return QKV_OK;
 }
 
@@ -281,8 +306,20 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   p.ws_lse = nullptr;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cache->key_block) {
+    // bf16 inputs split the cached keys when the caller gave the workspace for it.
+    const int n = dtype == QKV_BF16 ? channel_splits(cache, H_q, L_q) : 1;
+    const size_t need = split_workspace_bytes(cache, H_q, L_q, n);
+    if (n > 1 && workspace && workspace_bytes >= need && aligned16(workspace)) {
+      p.n_split = n;
+      p.ws_o = static_cast<float*>(workspace);
+      p.ws_lse = p.ws_o + static_cast<size_t>(n) * p.rows_all * cache->d;
+    }
     e = launch_attention_channel(p, cache->d, cache->bits, cache->key_block, st);
     if (e != cudaSuccess) return cuda_fail(e, "corrected_attention launch");
+    if (p.n_split > 1) {
+      e = launch_split_merge(p.ws_o, p.ws_lse, p.n_split, p.rows_all, cache->d, O, LSE, st);
+      if (e != cudaSuccess) return cuda_fail(e, "corrected_attention merge launch");
+    }
     return QKV_OK;
   }
   if (dtype == QKV_F32) {
@@ -355,8 +392,6 @@ QKV_API qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q,
   if (L_cur == 0 && cache->length == 0) return fail(QKV_ERR_INVALID_ARG, "no keys: empty cache and L_cur = 0");
   if (cache->length + L_cur >= 2147483647LL)
     return fail(QKV_ERR_UNSUPPORTED, "length + L_cur must be below 2^31 - 1");
-  if (cache->key_block)
-    return fail(QKV_ERR_UNSUPPORTED, "attention_fidelity: per-channel key blocks are not supported");
   if (!(std::isfinite(scale))) return fail(QKV_ERR_INVALID_ARG, "scale is not finite");
   if (L_q == 0) return QKV_OK;
   if (!Q || !stats) return fail(QKV_ERR_INVALID_ARG, "Q or stats is NULL");
@@ -377,6 +412,7 @@ QKV_API qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q,
   p.Lq = L_q; p.Lc = cache->length; p.Lcur = L_cur; p.capacity = cache->capacity;
   p.B = cache->B; p.Hq = H_q; p.Hkv = cache->H_kv; p.r = H_q / cache->H_kv;
   p.bits = cache->bits; p.group = cache->group; p.n_groups = cache->d / cache->group;
+  p.key_block = cache->key_block;
   p.correct = correct; p.causal = causal_cur;
   p.in_f32 = dtype == QKV_F32; p.meta_f16 = cache->meta_dtype == QKV_F16;
   p.scale = sc;

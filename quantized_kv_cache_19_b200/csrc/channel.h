@@ -26,8 +26,12 @@ cudaError_t launch_quantize_keys_channel(const ChanQuantParams& p, int in_dtype,
                                          int bits, cudaStream_t stream);
 
 // Corrected attention over a cache with per-channel key blocks of T positions (fp32 CUDA cores,
-// bf16 or fp32 inputs; O in the input type).
+// bf16 or fp32 inputs; O in the input type). With p.n_split > 1 (bf16 inputs only) the cached keys
+// are split over grid z and the normalised partials written to p.ws_o / p.ws_lse for the merge.
 cudaError_t launch_attention_channel(const AttnParams& p, int d, int bits, int T, cudaStream_t stream);
+// Query rows per CTA and keys per shared-memory tile of that kernel.
+int channel_rows_per_cta();
+int channel_tile_keys();
 
 // Correction term alone over per-channel key blocks: bias[B][Hq][Lq][Lc].
 cudaError_t launch_jensen_bias_channel(const BiasParams& p, int T, cudaStream_t stream);

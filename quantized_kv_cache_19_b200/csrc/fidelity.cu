@@ -101,11 +101,106 @@ __device__ __forceinline__ float4 load_key4(const void* base, int64_t elem, bool
   return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
 }
 
-template <int D>
+// One 4-channel chunk e of the key tile starting at k0: the reference key (K_ref, or K_cur past the
+// cache) and the dequantised key zp + step * code in fp32, plus the squared steps of the tile's
+// cached keys (per group and key; per channel for the block with per-channel keys).
+template <int D, bool kChan>
+__device__ __forceinline__ void fill_key_chunk(const FidelityParams& p, int e, int64_t k0, int64_t total,
+                                               int bh, bool f32, float* kr_s, float* kq_s, float* d2_s) {
+  constexpr int kPitch = D + 4;
+  const int kk = e / (D / 4), c4 = e - kk * (D / 4);
+  const int64_t key = k0 + kk;
+  float4 xr = make_float4(0.f, 0.f, 0.f, 0.f), xq = xr;
+  if (key < p.Lc) {
+    xr = load_key4(p.K_ref, (static_cast<int64_t>(bh) * p.Lc + key) * D + 4 * c4, f32);
+    const int64_t crow = static_cast<int64_t>(bh) * p.capacity + key;
+    const int g = (4 * c4) / p.group;
+    // (step, zero-point) of the 4 channels: one group's pair, or each channel's own pair
+    float st[4], zp[4];
+    if (kChan) {
+      const int64_t mi = ((static_cast<int64_t>(bh) * (p.capacity / p.key_block) + key / p.key_block) * D + 4 * c4) * 2;
+      if (p.meta_f16) {
+        const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __half*>(p.k_meta) + mi);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          st[i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] & 0xFFFFu)));
+          zp[i] = __half2float(__ushort_as_half(static_cast<unsigned short>(w[i] >> 16)));
+        }
+      } else {
+        const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(p.k_meta) + mi);
+        const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(p.k_meta) + mi + 4);
+        st[0] = a.x; zp[0] = a.y; st[1] = a.z; zp[1] = a.w;
+        st[2] = b.x; zp[2] = b.y; st[3] = b.z; zp[3] = b.w;
+      }
+    } else {
+      const int64_t mi = (crow * p.n_groups + g) * 2;
+      float s0, z0;
+      if (p.meta_f16) {
+        const __half* m = static_cast<const __half*>(p.k_meta) + mi;
+        s0 = __half2float(m[0]);
+        z0 = __half2float(m[1]);
+      } else {
+        const float* m = static_cast<const float*>(p.k_meta) + mi;
+        s0 = m[0];
+        z0 = m[1];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { st[i] = s0; zp[i] = z0; }
+    }
+    const uint8_t* cr = p.k_codes + crow * (D * p.bits / 8);
+    uint32_t c0, c1, c2, c3;
+    if (p.bits == 2) {
+      const uint32_t v = cr[c4];
+      c0 = v & 3u; c1 = (v >> 2) & 3u; c2 = (v >> 4) & 3u; c3 = v >> 6;
+    } else {
+      const uint32_t v = *reinterpret_cast<const uint16_t*>(cr + 2 * c4);
+      c0 = v & 15u; c1 = (v >> 4) & 15u; c2 = (v >> 8) & 15u; c3 = v >> 12;
+    }
+    xq = make_float4(fmaf(st[0], static_cast<float>(c0), zp[0]), fmaf(st[1], static_cast<float>(c1), zp[1]),
+                     fmaf(st[2], static_cast<float>(c2), zp[2]), fmaf(st[3], static_cast<float>(c3), zp[3]));
+    if (kChan) {
+      if (kk == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d2_s[4 * c4 + i] = st[i] * st[i];
+      }
+    } else if ((4 * c4) % p.group == 0) {
+      d2_s[kk * kMaxGroups + g] = st[0] * st[0];
+    }
+  } else if (key < total) {
+    xr = load_key4(p.K_cur, (static_cast<int64_t>(bh) * p.Lcur + (key - p.Lc)) * D + 4 * c4, f32);
+    xq = xr;
+  }
+  *reinterpret_cast<float4*>(kr_s + kk * kPitch + 4 * c4) = xr;
+  *reinterpret_cast<float4*>(kq_s + kk * kPitch + 4 * c4) = xq;
+}
+
+// Partial sums over channel quarter W of one row: (sum q_c^2 Delta_c^2, sum q_c^4 Delta_c^4), from
+// the row's q pairs and the block's squared steps, in fp32x2.
+template <int D, int W>
+__device__ __forceinline__ float2 tile_partial(const float2 (&q)[D / 2], const float* d2_s) {
+  const float2* d2p = reinterpret_cast<const float2*>(d2_s);
+  float2 s2 = make_float2(0.f, 0.f), s4 = s2;
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) {
+    const int c2 = (D / 8) * W + i;
+    const float2 qq = __fmul2_rn(q[c2], q[c2]);
+    const float2 t = __fmul2_rn(qq, d2p[c2]);
+    s2 = __fadd2_rn(s2, t);
+    s4 = __ffma2_rn(t, t, s4);
+  }
+  return make_float2(s2.x + s2.y, s4.x + s4.y);
+}
+
+// kChan: keys quantised per channel over blocks of p.key_block positions (a multiple of the 32-key
+// tile, so a tile lies in one block): the correction of a row is the same for all cached keys of a
+// tile, sum_c w_c Delta_c^2 (minus sum_c u_c Delta_c^4 for correct = 2), taken once per tile.
+template <int D, bool kChan>
 __global__ void __launch_bounds__(kThreadsF, 2) attention_fidelity_kernel(const FidelityParams p) {
   constexpr int kPitch = D + 4;
   __shared__ __align__(16) float tiles[2 * kKeysF * kPitch];
-  __shared__ float d2_s[kKeysF * kMaxGroups];             // squared steps of the cached keys
+  __shared__ __align__(8) float d2_s[kChan ? D : kKeysF * kMaxGroups];  // squared steps of the cached keys
+  __shared__ float2 part_s[kChan ? kSlices * kRowsF : 1];  // per-channel keys: partial corrections
   float* kr_s = tiles;                                    // reference (or current) keys
   float* kq_s = tiles + kKeysF * kPitch;                  // dequantised cached keys
   static_assert(2 * kKeysF * kPitch >= kSlices * kRowsF * (8 + 4 * kTop), "merge area");
@@ -144,7 +239,7 @@ __global__ void __launch_bounds__(kThreadsF, 2) attention_fidelity_kernel(const 
 #pragma unroll
       for (int k = 0; k < 4; ++k) q[4 * c8 + k] = make_float2(x[2 * k], x[2 * k + 1]);
     }
-    if (valid_row && p.correct) query_group_powers<D>(qrow, f32, G, p.wcoef, p.ucoef, w, u);
+    if (!kChan && valid_row && p.correct) query_group_powers<D>(qrow, f32, G, p.wcoef, p.ucoef, w, u);
   }
 
   Running ref{-INFINITY, 0.f, 0.f}, qnt{-INFINITY, 0.f, 0.f};
@@ -153,47 +248,39 @@ __global__ void __launch_bounds__(kThreadsF, 2) attention_fidelity_kernel(const 
   top_init(top_r);
   top_init(top_q);
 
-  const int row_codes = D * p.bits / 8;
   for (int64_t k0 = 0; k0 < total; k0 += kKeysF) {
     __syncthreads();
-    for (int e = t; e < kKeysF * (D / 4); e += kThreadsF) {
-      const int kk = e / (D / 4), c4 = e - kk * (D / 4);
-      const int64_t key = k0 + kk;
-      float4 xr = make_float4(0.f, 0.f, 0.f, 0.f), xq = xr;
-      if (key < p.Lc) {
-        xr = load_key4(p.K_ref, (static_cast<int64_t>(bh) * p.Lc + key) * D + 4 * c4, f32);
-        const int64_t crow = static_cast<int64_t>(bh) * p.capacity + key;
-        const int g = (4 * c4) / G;
-        float st, zp;
-        if (p.meta_f16) {
-          const __half* m = static_cast<const __half*>(p.k_meta) + (crow * NG + g) * 2;
-          st = __half2float(m[0]);
-          zp = __half2float(m[1]);
-        } else {
-          const float* m = static_cast<const float*>(p.k_meta) + (crow * NG + g) * 2;
-          st = m[0];
-          zp = m[1];
-        }
-        const uint8_t* cr = p.k_codes + crow * row_codes;
-        uint32_t c0, c1, c2, c3;
-        if (p.bits == 2) {
-          const uint32_t v = cr[c4];
-          c0 = v & 3u; c1 = (v >> 2) & 3u; c2 = (v >> 4) & 3u; c3 = v >> 6;
-        } else {
-          const uint32_t v = *reinterpret_cast<const uint16_t*>(cr + 2 * c4);
-          c0 = v & 15u; c1 = (v >> 4) & 15u; c2 = (v >> 8) & 15u; c3 = v >> 12;
-        }
-        xq = make_float4(fmaf(st, static_cast<float>(c0), zp), fmaf(st, static_cast<float>(c1), zp),
-                         fmaf(st, static_cast<float>(c2), zp), fmaf(st, static_cast<float>(c3), zp));
-        if ((4 * c4) % G == 0) d2_s[kk * kMaxGroups + g] = st * st;
-      } else if (key < total) {
-        xr = load_key4(p.K_cur, (static_cast<int64_t>(bh) * p.Lcur + (key - p.Lc)) * D + 4 * c4, f32);
-        xq = xr;
-      }
-      *reinterpret_cast<float4*>(kr_s + kk * kPitch + 4 * c4) = xr;
-      *reinterpret_cast<float4*>(kq_s + kk * kPitch + 4 * c4) = xq;
+    if (kChan) {
+#pragma unroll 1
+      for (int e = t; e < kKeysF * (D / 4); e += kThreadsF)
+        fill_key_chunk<D, kChan>(p, e, k0, total, bh, f32, kr_s, kq_s, d2_s);
+    } else {
+      for (int e = t; e < kKeysF * (D / 4); e += kThreadsF)
+        fill_key_chunk<D, kChan>(p, e, k0, total, bh, f32, kr_s, kq_s, d2_s);
     }
     __syncthreads();
+    // Per-channel keys: this row's correction for the tile, sum_c q_c^2 Delta_c^2 (and the fourth-
+    // order sum_c q_c^4 Delta_c^4), each warp over a quarter of the channels, combined in smem.
+    float tile_b = 0.f;
+    if (kChan && p.correct && k0 < p.Lc) {
+      float2 part;
+      switch (slice) {
+        case 0: part = tile_partial<D, 0>(q, d2_s); break;
+        case 1: part = tile_partial<D, 1>(q, d2_s); break;
+        case 2: part = tile_partial<D, 2>(q, d2_s); break;
+        default: part = tile_partial<D, 3>(q, d2_s); break;
+      }
+      part_s[slice * kRowsF + lane] = part;
+      __syncthreads();
+      float s2 = 0.f, s4 = 0.f;
+#pragma unroll
+      for (int w = 0; w < kSlices; ++w) {
+        s2 += part_s[w * kRowsF + lane].x;
+        s4 += part_s[w * kRowsF + lane].y;
+      }
+      tile_b = p.wcoef * s2;
+      if (p.correct == 2) tile_b = fmaf(-p.ucoef, s4, tile_b);
+    }
 #pragma unroll 1
     for (int kk = slice; kk < kKeysF; kk += kSlices) {
       const int64_t key = k0 + kk;
@@ -216,7 +303,9 @@ __global__ void __launch_bounds__(kThreadsF, 2) attention_fidelity_kernel(const 
         }
         sr = ((a0.x + a0.y) + (a1.x + a1.y)) * p.scale;
         sq = ((b0.x + b0.y) + (b1.x + b1.y)) * p.scale;
-        if (p.correct) {
+        if (kChan) {
+          sq -= tile_b;
+        } else if (p.correct) {
           float d2[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int g = 0; g < kMaxGroups; ++g)
@@ -323,7 +412,8 @@ template <int D>
 cudaError_t launch_fid(const FidelityParams& p, cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(p.r) * p.Lq;
   dim3 grid(static_cast<unsigned>((rows + kRowsF - 1) / kRowsF), static_cast<unsigned>(p.B * p.Hkv));
-  attention_fidelity_kernel<D><<<grid, kThreadsF, 0, stream>>>(p);
+  if (p.key_block) attention_fidelity_kernel<D, true><<<grid, kThreadsF, 0, stream>>>(p);
+  else attention_fidelity_kernel<D, false><<<grid, kThreadsF, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

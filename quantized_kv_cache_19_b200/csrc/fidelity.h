@@ -22,6 +22,7 @@ struct FidelityParams {
   int64_t Lq, Lc, Lcur, capacity;
   int B, Hq, Hkv, r;
   int bits, group, n_groups;
+  int key_block;          // 0: key groups per token; T: keys per channel over blocks of T positions
   int correct, causal;
   int in_f32, meta_f16;
   float scale;            // score scale (natural units)

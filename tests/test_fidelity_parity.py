@@ -45,20 +45,21 @@ def run_gpu(w, x, cache, correct, with_top=True):
     return st, top
 
 
-def oracle_rows(w, x, b, h, correct, rows):
+def oracle_rows(w, x, b, h, correct, rows, key_block=0):
     """The oracle on packed rows `rows` (head_in_group * Lq + i) of (batch b, KV head h)."""
     sub = sub_problem(x, w, b, h)
     d = w.d
+    group = 1 if key_block else w.group
     if w.Lc:
-        c = oracle.build_cache(sub["K_src"], sub["V_src"], w.bits, w.group, w.meta)
+        c = oracle.build_cache(sub["K_src"], sub["V_src"], w.bits, w.group, w.meta, key_block=key_block)
         kh, _, ks = oracle.cache_rows(c, 0, 0)
         k_ref = sub["K_src"][0, 0]
     else:
-        kh, ks, k_ref = np.zeros((0, d)), np.zeros((0, w.n_groups)), np.zeros((0, d))
+        kh, ks, k_ref = np.zeros((0, d)), np.zeros((0, d // group)), np.zeros((0, d))
     k_cur = sub["K_cur"][0, 0] if w.Lcur else np.zeros((0, d))
     rows = np.asarray(rows)
     q = sub["Q"][0][rows // w.Lq, rows % w.Lq]
-    return oracle.fidelity_rows(q, rows % w.Lq, k_ref, kh, ks, w.group, k_cur, correct, w.causal,
+    return oracle.fidelity_rows(q, rows % w.Lq, k_ref, kh, ks, group, k_cur, correct, w.causal,
                                 1.0 / math.sqrt(d), w.Lq, return_scores=True)
 
 
@@ -113,14 +114,25 @@ def compare(st, top, f, what, lse_tol=LSE_TOL):
     return errs
 
 
-def check_all_rows(w, correct, seed=None):
+def chan_cache(w, K, V, T):
+    cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc), w.meta,
+                        device=K.device, key_block=T)
+    if w.Lc:
+        api.kv_quantize_append(cache, K, V)
+    return cache
+
+
+def check_all_rows(w, correct, seed=None, key_block=0):
     x = make_inputs(w, device="cuda", seed=seed)
-    cache = build_gpu_cache(w, x["K_src"], x["V_src"])
+    if key_block:
+        cache = chan_cache(w, x["K_src"], x["V_src"], key_block)
+    else:
+        cache = build_gpu_cache(w, x["K_src"], x["V_src"])
     st, top = run_gpu(w, x, cache, correct)
     rows = np.arange(w.rows_per_kv_head)
     for b in range(w.B):
         for h in range(w.Hkv):
-            f = oracle_rows(w, x, b, h, correct, rows)
+            f = oracle_rows(w, x, b, h, correct, rows, key_block)
             s, t = gpu_rows(w, st, top, b, h, rows)
             compare(s, t, f, f"{w.name} b{b} h{h} correct={correct}")
     assert api.device_status() == 0
@@ -228,3 +240,23 @@ def test_correction_restores_cached_mass_full_bf16_int2():
             assert abs(g[:, 3].mean() - f["mass_q"].mean()) < 1e-5
             assert abs(g[:, 4].mean() - f["kl"].mean()) < 1e-4
             assert abs(g[:, 5].mean() - f["top1_agree"].mean()) < 0.01
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "bf16_int2", "long_video", "prefill_gqa"])
+@pytest.mark.parametrize("correct", [0, 1, 2])
+def test_every_row_per_channel_keys(name, correct):
+    """Caches with per-channel key blocks (32 positions): the correction uses each key's block steps."""
+    check_all_rows(SMALL[name], correct, key_block=32)
+
+
+def test_full_size_sampled_rows_per_channel_keys():
+    w = WORKLOADS["bf16_int2"]
+    x = make_inputs(w, device="cuda")
+    cache = chan_cache(w, x["K_src"], x["V_src"], 32)
+    st, top = run_gpu(w, x, cache, 1)
+    rows = sample_rows(w, 64).numpy()
+    for b, h in [(0, 1), (0, 14)]:
+        f = oracle_rows(w, x, b, h, 1, rows, key_block=32)
+        s, t = gpu_rows(w, st, top, b, h, rows)
+        compare(s, t, f, f"bf16_int2 per-channel b{b} h{h}", lse_tol=FULL_LSE_TOL)
+    assert api.device_status() == 0

@@ -71,13 +71,17 @@ def oracle_head(w, sub, T, correct, rows=None):
                                       causal=w.causal, scale=1.0 / math.sqrt(w.d), rows=rows)
 
 
-def check_every_row(w, T, correct, noalloc=False):
+def check_every_row(w, T, correct, mode="auto"):
+    """mode: "auto" (key split when the shape asks for it), "unsplit" (no workspace) or "noalloc"."""
     x = make_inputs(w, device="cuda")
     cache = build_chan_cache(w, x["K_src"], x["V_src"], T)
     Kc = x["K_cur"] if w.Lcur else None
     Vc = x["V_cur"] if w.Lcur else None
-    fn = api.corrected_attention_noalloc if noalloc else api.corrected_attention
-    O, LSE = fn(x["Q"], cache, Kc, Vc, correct=correct, causal=w.causal)
+    if mode == "noalloc":
+        O, LSE = api.corrected_attention_noalloc(x["Q"], cache, Kc, Vc, correct=correct, causal=w.causal)
+    else:
+        O, LSE = api.corrected_attention(x["Q"], cache, Kc, Vc, correct=correct, causal=w.causal,
+                                         workspace="auto" if mode == "auto" else None)
     torch.cuda.synchronize()
     r = w.Hq // w.Hkv
     for b in range(w.B):
@@ -111,10 +115,26 @@ def test_attention_edge_cases():
 
 
 def test_noalloc_entry_point_serves_per_channel_keys():
+    """The allocation-free entry point runs per-channel caches unsplit: the same result as the
+    workspace-free call."""
     w = SMALL["prefill_gqa"].with_(Lq=4, Lcur=4)
-    O1, L1 = check_every_row(w, 32, 1, noalloc=True)
-    O2, L2 = check_every_row(w, 32, 1)
+    O1, L1 = check_every_row(w, 32, 1, mode="noalloc")
+    O2, L2 = check_every_row(w, 32, 1, mode="unsplit")
     assert torch.equal(O1, O2) and torch.equal(L1, L2)
+
+
+@pytest.mark.parametrize("Lq,causal", [(1, True), (4, False), (16, True)])
+def test_key_split_every_row_and_against_unsplit(Lq, causal):
+    """Few query rows per KV head: the bf16 path splits the cached keys over CTAs and merges the
+    partials. Every row against the oracle, and the split against the unsplit kernel."""
+    w = SMALL["prefill_gqa"].with_(Lq=Lq, Lcur=Lq, Lc=32 * 40 + 9, causal=causal)
+    cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc), w.meta, key_block=32)
+    cache.length = w.Lc
+    assert api.attention_workspace_bytes(cache, w.Hq, w.Lq, w.Lcur) > 0
+    O1, L1 = check_every_row(w, 32, 1, mode="auto")
+    O2, L2 = check_every_row(w, 32, 1, mode="unsplit")
+    compare(np32(O1).astype(np.float64), np32(O2).astype(np.float64), np32(L1).astype(np.float64),
+            np32(L2).astype(np.float64), f"per-channel split vs unsplit Lq={Lq}")
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "bf16_int2", "long_video"])
