@@ -6,9 +6,11 @@
 // Jensen 偏差", sections 方法 / 為何校正有效): scores q . x_hat * scale over the dequantised cache
 // minus the Jensen term b, then over the current chunk, one online softmax, O and LSE.
 //
-// One CTA of 128 threads per (128 packed query rows, batch * KV head); one thread per query row.
-// Keys are staged 32 at a time in shared memory as fp32 (cached keys dequantised with one fp32
-// FMA, zp + step * code), and every thread walks them in order.
+// One CTA of 256 threads per (128 packed query rows, batch * KV head); two threads per query row,
+// one on the even and one on the odd keys of each tile. Keys are staged 32 at a time in shared
+// memory as fp32 (cached keys dequantised with one fp32 FMA, zp + step * code); a row's q is read
+// from shared memory in 16-byte pieces, keys and values as broadcasts, and the dot products and the
+// P.V update use packed fp32x2 FMAs.
 //
 // The same kernel serves caches whose keys are quantised per channel along tokens (KIVI's key
 // grouping, agents-report.net, section 跨主題對比分析; hotelren.com blog, section 3.1): every T
@@ -27,12 +29,8 @@ namespace qkv {
 namespace {
 
 constexpr int kRows = 128;
+constexpr int kThreads = 2 * kRows;   // two threads per query row
 constexpr int kKT = 32;         // keys per shared-memory tile
-
-__device__ __forceinline__ int code_at(const uint8_t* row, int c, int bits) {
-  const int bit = c * bits;
-  return (row[bit >> 3] >> (bit & 7)) & ((1 << bits) - 1);
-}
 
 template <bool kF32In>
 __device__ __forceinline__ float ld_in(const void* base, int64_t i) {
@@ -40,46 +38,72 @@ __device__ __forceinline__ float ld_in(const void* base, int64_t i) {
   return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
 }
 
+// Codes of 4 consecutive channels c4*4 .. c4*4+3 of a packed row.
+__device__ __forceinline__ void codes4(const uint8_t* row, int c4, int bits, float (&c)[4]) {
+  if (bits == 2) {
+    const uint32_t v = row[c4];
+    c[0] = static_cast<float>(v & 3u); c[1] = static_cast<float>((v >> 2) & 3u);
+    c[2] = static_cast<float>((v >> 4) & 3u); c[3] = static_cast<float>(v >> 6);
+  } else {
+    const uint32_t v = *reinterpret_cast<const uint16_t*>(row + 2 * c4);
+    c[0] = static_cast<float>(v & 15u); c[1] = static_cast<float>((v >> 4) & 15u);
+    c[2] = static_cast<float>((v >> 8) & 15u); c[3] = static_cast<float>(v >> 12);
+  }
+}
+
+template <bool kF32In>
+__device__ __forceinline__ float4 ld_in4(const void* base, int64_t i) {
+  if (kF32In) return *reinterpret_cast<const float4*>(static_cast<const float*>(base) + i);
+  const uint2 u = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + i);
+  return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+}
+
 // kChan: keys quantised per channel over blocks of T positions (meta [BH][capacity/T][D][2]);
 // otherwise per token in groups of p.group channels. kF32In: Q, K_cur, V_cur and O are fp32 (else bf16).
+// Two threads per query row (threads t and t + 128): each takes the even or the odd keys of every
+// 32-key tile with its own running max, sum and O, merged through shared memory at the end.
 template <int D, bool kChan, bool kF32In>
-__global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p, int bits, int T) {
+__global__ void __launch_bounds__(kThreads) attention_f32_kernel(const AttnParams p, int bits, int T) {
+  constexpr int kPitch = D + 4;                 // 16-byte rows; 8 lanes' rows hit distinct banks
   extern __shared__ float sm[];
-  float* q_s = sm;                              // [128][D + 1]
-  float* k_s = q_s + kRows * (D + 1);           // [kKT][D]
+  float* q_s = sm;                              // [128][kPitch]
+  float* k_s = q_s + kRows * kPitch;            // [kKT][D]
   float* v_s = k_s + kKT * D;                   // [kKT][D]
   float* d2_s = v_s + kKT * D;                  // [kKT][4]; per-channel keys: [D] squared steps
   const int t = threadIdx.x;
-  const int m_tile = blockIdx.x;
+  const int rt = t & (kRows - 1);               // row within the tile
+  const int par = t / kRows;                    // key parity this thread takes
   const int bh = blockIdx.y;
   const int b = bh / p.Hkv;
   const int h = bh - b * p.Hkv;
   const int64_t rows_total = static_cast<int64_t>(p.r) * p.Lq;
-  const int64_t R = static_cast<int64_t>(m_tile) * kRows + t;
+  const int64_t R = static_cast<int64_t>(blockIdx.x) * kRows + rt;
   const bool valid_row = R < rows_total;
   const int64_t hq = static_cast<int64_t>(h) * p.r + (valid_row ? R / p.Lq : 0);
   const int64_t qi = valid_row ? R % p.Lq : 0;
   const int64_t out_row = (static_cast<int64_t>(b) * p.Hq + hq) * p.Lq + qi;
   const float scale = p.scale_log2 * 0.69314718055994530942f;   // natural units here
   const float wcoef = p.wcoef_log2 * 0.69314718055994530942f;
+  const float ucoef = p.ucoef_log2 * 0.69314718055994530942f;
   const int G = p.group, NG = p.n_groups;
   const int row_codes = D * bits / 8;
 
-  const float ucoef = p.ucoef_log2 * 0.69314718055994530942f;
   float w[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
   float u[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
   const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * (kF32In ? 4 : 2);
-  if (valid_row) {
-    if (!kChan && p.correct) query_group_powers<D>(qrow, kF32In, G, wcoef, ucoef, w, u);
-    for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = ld_in<kF32In>(qrow, c);
-  } else {
-    for (int c = 0; c < D; ++c) q_s[t * (D + 1) + c] = 0.f;
+  if (!kChan && valid_row && p.correct) query_group_powers<D>(qrow, kF32In, G, wcoef, ucoef, w, u);
+  if (par == 0) {
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+      const float4 x = valid_row ? ld_in4<kF32In>(qrow, 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(q_s + rt * kPitch + 4 * c4) = x;
+    }
   }
-  float o[D];
+  float2 o[D / 2];
 #pragma unroll
-  for (int c = 0; c < D; ++c) o[c] = 0.f;
+  for (int c = 0; c < D / 2; ++c) o[c] = make_float2(0.f, 0.f);
   float m = -INFINITY, l = 0.f;
   const int64_t lim_cur = p.causal ? qi + (p.Lcur - p.Lq) + 1 : p.Lcur;   // current keys this row sees
+  const float4* q4 = reinterpret_cast<const float4*>(q_s + rt * kPitch);
 
   // Keys [k_begin, total) of this CTA. With a split over the cached keys (n_split > 1, grid z),
   // split z takes the 32-key cached tiles [z T / n, (z+1) T / n) and the last split also the
@@ -93,102 +117,176 @@ __global__ void __launch_bounds__(kRows) attention_f32_kernel(const AttnParams p
   }
   for (int64_t k0 = k_begin; k0 < total; k0 += kKT) {
     __syncthreads();
-    for (int e = t; e < kKT * D; e += kRows) {
-      const int kk = e / D, c = e % D;
+    for (int e = t; e < kKT * (D / 4); e += kThreads) {
+      const int kk = e / (D / 4), c4 = e % (D / 4);
       const int64_t key = k0 + kk;
-      float kv = 0.f, vv = 0.f;
+      float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
       if (key < p.Lc) {
         const int64_t row = static_cast<int64_t>(bh) * p.capacity + key;
-        const int g = c / G;
-        // key meta: per (token, group), or per (block of T tokens, channel)
-        const int64_t kmi = kChan ? ((static_cast<int64_t>(bh) * (p.capacity / T) + key / T) * D + c) * 2
-                                  : (row * NG + g) * 2;
-        float ks, kz, vs, vz;
-        if (p.meta_f16) {
-          const __half* km = static_cast<const __half*>(p.k_meta) + kmi;
-          const __half* vm = static_cast<const __half*>(p.v_meta) + (row * NG + g) * 2;
-          ks = __half2float(km[0]); kz = __half2float(km[1]);
-          vs = __half2float(vm[0]); vz = __half2float(vm[1]);
-        } else {
-          const float* km = static_cast<const float*>(p.k_meta) + kmi;
-          const float* vm = static_cast<const float*>(p.v_meta) + (row * NG + g) * 2;
-          ks = km[0]; kz = km[1]; vs = vm[0]; vz = vm[1];
-        }
-        kv = fmaf(ks, static_cast<float>(code_at(p.k_codes + row * row_codes, c, bits)), kz);
-        vv = fmaf(vs, static_cast<float>(code_at(p.v_codes + row * row_codes, c, bits)), vz);
+        const int g = (4 * c4) / G;
+        const int64_t vmi = (row * NG + g) * 2;
+        float ks[4], kz[4], vs, vz;
         if (kChan) {
-          if (kk == 0) d2_s[c] = ks * ks;        // the tile lies in one key block (T % 32 == 0)
-        } else if (c % G == 0) {
-          d2_s[kk * 4 + g] = ks * ks;
+          const int64_t kmi = ((static_cast<int64_t>(bh) * (p.capacity / T) + key / T) * D + 4 * c4) * 2;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (p.meta_f16) {
+              ks[i] = __half2float(static_cast<const __half*>(p.k_meta)[kmi + 2 * i]);
+              kz[i] = __half2float(static_cast<const __half*>(p.k_meta)[kmi + 2 * i + 1]);
+            } else {
+              ks[i] = static_cast<const float*>(p.k_meta)[kmi + 2 * i];
+              kz[i] = static_cast<const float*>(p.k_meta)[kmi + 2 * i + 1];
+            }
+          }
+        } else {
+          const int64_t kmi = (row * NG + g) * 2;
+          float s0, z0;
+          if (p.meta_f16) {
+            s0 = __half2float(static_cast<const __half*>(p.k_meta)[kmi]);
+            z0 = __half2float(static_cast<const __half*>(p.k_meta)[kmi + 1]);
+          } else {
+            s0 = static_cast<const float*>(p.k_meta)[kmi];
+            z0 = static_cast<const float*>(p.k_meta)[kmi + 1];
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) { ks[i] = s0; kz[i] = z0; }
+        }
+        if (p.meta_f16) {
+          vs = __half2float(static_cast<const __half*>(p.v_meta)[vmi]);
+          vz = __half2float(static_cast<const __half*>(p.v_meta)[vmi + 1]);
+        } else {
+          vs = static_cast<const float*>(p.v_meta)[vmi];
+          vz = static_cast<const float*>(p.v_meta)[vmi + 1];
+        }
+        float kc[4], vc[4];
+        codes4(p.k_codes + row * row_codes, c4, bits, kc);
+        codes4(p.v_codes + row * row_codes, c4, bits, vc);
+        kv = make_float4(fmaf(ks[0], kc[0], kz[0]), fmaf(ks[1], kc[1], kz[1]),
+                         fmaf(ks[2], kc[2], kz[2]), fmaf(ks[3], kc[3], kz[3]));
+        vv = make_float4(fmaf(vs, vc[0], vz), fmaf(vs, vc[1], vz), fmaf(vs, vc[2], vz), fmaf(vs, vc[3], vz));
+        if (kChan) {
+          if (kk == 0) {                          // the tile lies in one key block (T % 32 == 0)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d2_s[4 * c4 + i] = ks[i] * ks[i];
+          }
+        } else if ((4 * c4) % G == 0) {
+          d2_s[kk * 4 + g] = ks[0] * ks[0];
         }
       } else if (key < total) {
         const int64_t row = static_cast<int64_t>(bh) * p.Lcur + (key - p.Lc);
-        kv = ld_in<kF32In>(p.K_cur, row * D + c);
-        vv = ld_in<kF32In>(p.V_cur, row * D + c);
+        kv = ld_in4<kF32In>(p.K_cur, row * D + 4 * c4);
+        vv = ld_in4<kF32In>(p.V_cur, row * D + 4 * c4);
       }
-      k_s[kk * D + c] = kv;
-      v_s[kk * D + c] = vv;
+      *reinterpret_cast<float4*>(k_s + kk * D + 4 * c4) = kv;
+      *reinterpret_cast<float4*>(v_s + kk * D + 4 * c4) = vv;
     }
     __syncthreads();
     // Per-channel keys: the tile's correction for this row, sum_c w_c Delta_c^2 (minus the fourth-
     // order term sum_c u_c Delta_c^4 when correct = 2), one pass over the block's squared steps.
     float tile_b = 0.f;
     if (kChan && p.correct && k0 < p.Lc) {
-      for (int c = 0; c < D; ++c) {
-        const float q2 = q_s[t * (D + 1) + c] * q_s[t * (D + 1) + c];
-        const float d2 = d2_s[c];
-        tile_b = fmaf(wcoef * q2, d2, tile_b);
-        if (p.correct == 2) tile_b = fmaf(-ucoef * (q2 * q2), d2 * d2, tile_b);
+      float2 s2 = make_float2(0.f, 0.f), s4 = s2;
+      const float4* d4 = reinterpret_cast<const float4*>(d2_s);
+#pragma unroll 4
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 x = q4[c4], d = d4[c4];
+        const float2 t0 = __fmul2_rn(__fmul2_rn(make_float2(x.x, x.y), make_float2(x.x, x.y)), make_float2(d.x, d.y));
+        const float2 t1 = __fmul2_rn(__fmul2_rn(make_float2(x.z, x.w), make_float2(x.z, x.w)), make_float2(d.z, d.w));
+        s2 = __fadd2_rn(s2, __fadd2_rn(t0, t1));
+        s4 = __ffma2_rn(t0, t0, __ffma2_rn(t1, t1, s4));
       }
+      tile_b = wcoef * (s2.x + s2.y);
+      if (p.correct == 2) tile_b = fmaf(-ucoef, s4.x + s4.y, tile_b);
     }
-    for (int kk = 0; kk < kKT; ++kk) {
+    for (int kk = par; kk < kKT; kk += 2) {
       const int64_t key = k0 + kk;
       if (key >= total) break;
       const bool cached = key < p.Lc;
       if (!cached && (key - p.Lc) >= lim_cur) continue;
-      float s = 0.f;
-      for (int c = 0; c < D; ++c) s = fmaf(q_s[t * (D + 1) + c], k_s[kk * D + c], s);
-      s *= scale;
+      const float4* k4 = reinterpret_cast<const float4*>(k_s + kk * D);
+      float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 x = q4[c4], y = k4[c4];
+        a0 = __ffma2_rn(make_float2(x.x, x.y), make_float2(y.x, y.y), a0);
+        a1 = __ffma2_rn(make_float2(x.z, x.w), make_float2(y.z, y.w), a1);
+      }
+      float s = ((a0.x + a0.y) + (a1.x + a1.y)) * scale;
       if (kChan) {
         if (cached) s -= tile_b;
       } else if (cached && p.correct) {
         float d2[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
-        for (int g = 0; g < NG; ++g) d2[g] = d2_s[kk * 4 + g];
+#pragma unroll
+        for (int g = 0; g < kMaxGroups; ++g)
+          if (g < NG) d2[g] = d2_s[kk * 4 + g];
         s -= jensen_term(w, d2, NG);
         if (p.correct == 2) {
-          for (int g = 0; g < NG; ++g) s = fmaf(u[g], d2[g] * d2[g], s);
+#pragma unroll
+          for (int g = 0; g < kMaxGroups; ++g)
+            if (g < NG) s = fmaf(u[g], d2[g] * d2[g], s);
         }
       }
       if (s > m) {
         const float a = expf(m - s);       // 0 when m = -inf
         l *= a;
+        const float2 a2 = make_float2(a, a);
 #pragma unroll
-        for (int c = 0; c < D; ++c) o[c] *= a;
+        for (int c = 0; c < D / 2; ++c) o[c] = __fmul2_rn(o[c], a2);
         m = s;
       }
       const float pk = expf(s - m);
       l += pk;
+      const float2 p2 = make_float2(pk, pk);
+      const float4* v4 = reinterpret_cast<const float4*>(v_s + kk * D);
 #pragma unroll
-      for (int c = 0; c < D; ++c) o[c] = fmaf(pk, v_s[kk * D + c], o[c]);
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 y = v4[c4];
+        o[2 * c4] = __ffma2_rn(p2, make_float2(y.x, y.y), o[2 * c4]);
+        o[2 * c4 + 1] = __ffma2_rn(p2, make_float2(y.z, y.w), o[2 * c4 + 1]);
+      }
     }
   }
-  if (valid_row && p.n_split > 1) {
+  // Merge the odd-key half of each row into the even-key half (q_s is free now).
+  __syncthreads();
+  float* mg = q_s + rt * kPitch;                // [D] partial O, then m and l
+  if (par == 1) {
+#pragma unroll
+    for (int c = 0; c < D / 2; ++c) *reinterpret_cast<float2*>(mg + 2 * c) = o[c];
+    mg[D] = m;
+    mg[D + 1] = l;
+  }
+  __syncthreads();
+  if (par == 1 || !valid_row) return;
+  {
+    const float m2 = mg[D], l2 = mg[D + 1];
+    const float mn = fmaxf(m, m2);
+    if (mn != -INFINITY) {
+      const float f1 = expf(m - mn), f2 = expf(m2 - mn);
+      l = l * f1 + l2 * f2;
+      const float2 f1v = make_float2(f1, f1), f2v = make_float2(f2, f2);
+#pragma unroll
+      for (int c = 0; c < D / 2; ++c)
+        o[c] = __ffma2_rn(f2v, *reinterpret_cast<const float2*>(mg + 2 * c), __fmul2_rn(o[c], f1v));
+      m = mn;
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  if (p.n_split > 1) {
     const int64_t prow = static_cast<int64_t>(blockIdx.z) * p.rows_all + out_row;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
     float* orow = p.ws_o + prow * D;
 #pragma unroll
-    for (int c = 0; c < D; ++c) orow[c] = o[c] * inv;
+    for (int c = 0; c < D / 2; ++c) *reinterpret_cast<float2*>(orow + 2 * c) = make_float2(o[c].x * inv, o[c].y * inv);
     p.ws_lse[prow] = l > 0.f ? m + logf(l) : -INFINITY;
-  } else if (valid_row) {
-    const float inv = l > 0.f ? 1.f / l : 0.f;
+  } else {
     if (kF32In) {
       float* orow = static_cast<float*>(p.O) + out_row * D;
 #pragma unroll
-      for (int c = 0; c < D; ++c) orow[c] = o[c] * inv;
+      for (int c = 0; c < D / 2; ++c) *reinterpret_cast<float2*>(orow + 2 * c) = make_float2(o[c].x * inv, o[c].y * inv);
     } else {
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.O) + out_row * D;
 #pragma unroll
-      for (int c = 0; c < D; ++c) orow[c] = __float2bfloat16_rn(o[c] * inv);
+      for (int c = 0; c < D / 2; ++c)
+        *reinterpret_cast<__nv_bfloat162*>(orow + 2 * c) = __floats2bfloat162_rn(o[c].x * inv, o[c].y * inv);
     }
     p.LSE[out_row] = l > 0.f ? m + logf(l) : -INFINITY;
   }
@@ -240,7 +338,7 @@ __global__ void __launch_bounds__(256) jensen_bias_channel_kernel(const BiasPara
 
 template <int D, bool kChan, bool kF32In>
 cudaError_t launch_f32(const AttnParams& p, int bits, int T, cudaStream_t stream) {
-  const size_t smem = (kRows * (D + 1) + 2 * kKT * D + (kChan ? D : kKT * 4)) * sizeof(float);
+  const size_t smem = (kRows * (D + 4) + 2 * kKT * D + (kChan ? D : kKT * 4)) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(attention_f32_kernel<D, kChan, kF32In>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -248,7 +346,7 @@ cudaError_t launch_f32(const AttnParams& p, int bits, int T, cudaStream_t stream
   const int64_t rows = static_cast<int64_t>(p.r) * p.Lq;
   dim3 grid(static_cast<unsigned>((rows + kRows - 1) / kRows), static_cast<unsigned>(p.B * p.Hkv),
             static_cast<unsigned>(p.n_split > 1 ? p.n_split : 1));
-  attention_f32_kernel<D, kChan, kF32In><<<grid, kRows, smem, stream>>>(p, bits, T);
+  attention_f32_kernel<D, kChan, kF32In><<<grid, kThreads, smem, stream>>>(p, bits, T);
   return cudaGetLastError();
 }
 
