@@ -58,6 +58,23 @@ __device__ __forceinline__ float4 ld_in4(const void* base, int64_t i) {
   return make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
 }
 
+// A cached key's score minus the correction from its per-group squared steps d2[g] (plus the
+// fourth-order term u_g d2_g^2 when correct = 2).
+__device__ __forceinline__ float corrected(float s, const float (&w)[kMaxGroups], const float (&u)[kMaxGroups],
+                                           const float* d2s, int NG, int correct) {
+  float d2[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int g = 0; g < kMaxGroups; ++g)
+    if (g < NG) d2[g] = d2s[g];
+  s -= jensen_term(w, d2, NG);
+  if (correct == 2) {
+#pragma unroll
+    for (int g = 0; g < kMaxGroups; ++g)
+      if (g < NG) s = fmaf(u[g], d2[g] * d2[g], s);
+  }
+  return s;
+}
+
 // kChan: keys quantised per channel over blocks of T positions (meta [BH][capacity/T][D][2]);
 // otherwise per token in groups of p.group channels. kF32In: Q, K_cur, V_cur and O are fp32 (else bf16).
 // Two threads per query row (threads t and t + 128): each takes the even or the odd keys of every
@@ -92,10 +109,18 @@ __global__ void __launch_bounds__(kThreads) attention_f32_kernel(const AttnParam
   float u[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
   const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * (kF32In ? 4 : 2);
   if (!kChan && valid_row && p.correct) query_group_powers<D>(qrow, kF32In, G, wcoef, ucoef, w, u);
+  // The row's q in shared memory: fp32, or for bf16 inputs as bf16 (exact), 8 channels per 16 bytes.
   if (par == 0) {
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-      const float4 x = valid_row ? ld_in4<kF32In>(qrow, 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(q_s + rt * kPitch + 4 * c4) = x;
+    if (kF32In) {
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 x = valid_row ? ld_in4<kF32In>(qrow, 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(q_s + rt * kPitch + 4 * c4) = x;
+      }
+    } else {
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint4 v = valid_row ? reinterpret_cast<const uint4*>(qrow)[c8] : make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(q_s + rt * kPitch)[c8] = v;
+      }
     }
   }
   float2 o[D / 2];
@@ -103,7 +128,8 @@ __global__ void __launch_bounds__(kThreads) attention_f32_kernel(const AttnParam
   for (int c = 0; c < D / 2; ++c) o[c] = make_float2(0.f, 0.f);
   float m = -INFINITY, l = 0.f;
   const int64_t lim_cur = p.causal ? qi + (p.Lcur - p.Lq) + 1 : p.Lcur;   // current keys this row sees
-  const float4* q4 = reinterpret_cast<const float4*>(q_s + rt * kPitch);
+  const float4* q4 = reinterpret_cast<const float4*>(q_s + rt * kPitch);      // fp32 q
+  const uint4* qb8 = reinterpret_cast<const uint4*>(q_s + rt * kPitch);       // bf16 q
 
   // Keys [k_begin, total) of this CTA. With a split over the cached keys (n_split > 1, grid z),
   // split z takes the 32-key cached tiles [z T / n, (z+1) T / n) and the last split also the
@@ -187,9 +213,16 @@ __global__ void __launch_bounds__(kThreads) attention_f32_kernel(const AttnParam
     if (kChan && p.correct && k0 < p.Lc) {
       float2 s2 = make_float2(0.f, 0.f), s4 = s2;
       const float4* d4 = reinterpret_cast<const float4*>(d2_s);
-#pragma unroll 4
+#pragma unroll
       for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 x = q4[c4], d = d4[c4];
+        float4 x;
+        if (kF32In) {
+          x = q4[c4];
+        } else {
+          const uint2 u = reinterpret_cast<const uint2*>(qb8)[c4];
+          x = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+        }
+        const float4 d = d4[c4];
         const float2 t0 = __fmul2_rn(__fmul2_rn(make_float2(x.x, x.y), make_float2(x.x, x.y)), make_float2(d.x, d.y));
         const float2 t1 = __fmul2_rn(__fmul2_rn(make_float2(x.z, x.w), make_float2(x.z, x.w)), make_float2(d.z, d.w));
         s2 = __fadd2_rn(s2, __fadd2_rn(t0, t1));
@@ -205,26 +238,29 @@ __global__ void __launch_bounds__(kThreads) attention_f32_kernel(const AttnParam
       if (!cached && (key - p.Lc) >= lim_cur) continue;
       const float4* k4 = reinterpret_cast<const float4*>(k_s + kk * D);
       float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+      if (kF32In) {
 #pragma unroll
-      for (int c4 = 0; c4 < D / 4; ++c4) {
-        const float4 x = q4[c4], y = k4[c4];
-        a0 = __ffma2_rn(make_float2(x.x, x.y), make_float2(y.x, y.y), a0);
-        a1 = __ffma2_rn(make_float2(x.z, x.w), make_float2(y.z, y.w), a1);
+        for (int c4 = 0; c4 < D / 4; ++c4) {
+          const float4 x = q4[c4], y = k4[c4];
+          a0 = __ffma2_rn(make_float2(x.x, x.y), make_float2(y.x, y.y), a0);
+          a1 = __ffma2_rn(make_float2(x.z, x.w), make_float2(y.z, y.w), a1);
+        }
+      } else {
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          const uint4 u = qb8[c8];
+          const float4 y = k4[2 * c8], z = k4[2 * c8 + 1];
+          a0 = __ffma2_rn(make_float2(bf16_lo(u.x), bf16_hi(u.x)), make_float2(y.x, y.y), a0);
+          a1 = __ffma2_rn(make_float2(bf16_lo(u.y), bf16_hi(u.y)), make_float2(y.z, y.w), a1);
+          a0 = __ffma2_rn(make_float2(bf16_lo(u.z), bf16_hi(u.z)), make_float2(z.x, z.y), a0);
+          a1 = __ffma2_rn(make_float2(bf16_lo(u.w), bf16_hi(u.w)), make_float2(z.z, z.w), a1);
+        }
       }
       float s = ((a0.x + a0.y) + (a1.x + a1.y)) * scale;
       if (kChan) {
         if (cached) s -= tile_b;
       } else if (cached && p.correct) {
-        float d2[kMaxGroups] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int g = 0; g < kMaxGroups; ++g)
-          if (g < NG) d2[g] = d2_s[kk * 4 + g];
-        s -= jensen_term(w, d2, NG);
-        if (p.correct == 2) {
-#pragma unroll
-          for (int g = 0; g < kMaxGroups; ++g)
-            if (g < NG) s = fmaf(u[g], d2[g] * d2[g], s);
-        }
+        s = corrected(s, w, u, d2_s + kk * 4, NG, p.correct);
       }
       if (s > m) {
         const float a = expf(m - s);       // 0 when m = -inf
