@@ -146,7 +146,9 @@ qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H
  *                 key split. Calls on one stream may reuse it; concurrent calls need their own.
  * L_cur = 0 and cache->length = 0 together are rejected (no keys at all).
  * A cache with per-channel keys (key_block > 0) is served by an fp32 CUDA-core kernel for bf16 and
- * fp32 inputs alike; it uses no workspace (corrected_attention_workspace_bytes() gives 0).
+ * fp32 inputs alike. With bf16 inputs it splits the cached keys over CTAs for decode-sized query
+ * chunks (when the unsplit grid would leave more than half of the SMs idle) and then uses the
+ * workspace the same way; fp32 inputs run unsplit and ignore the workspace.
  */
 qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
                                const qkv_cache* cache, const void* K_cur, const void* V_cur,
@@ -162,7 +164,7 @@ qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_
  * that loads the library, kept until the process exits. No call allocates or frees memory.
  *  - A shape whose split needs more than 8 MiB of scratch (corrected_attention_workspace_bytes()
  *    larger than 8 MiB) is rejected with QKV_ERR_UNSUPPORTED; corrected_attention with a workspace
- *    handles it.
+ *    handles it. Caches with per-channel keys (key_block > 0) run unsplit here and need no scratch.
  *  - The first call on a device that needs the scratch looks up the array's device address (with
  *    that device current); make that first call before any stream capture.
  *  - All calls share the one array: every value a call reads from it was written by the same call,
