@@ -3,10 +3,15 @@ INT2 cache plus the unquantised chunk, then quantise-append of the finished chun
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Prints ONE JSON line (rank 0). `value` is attention TFLOP/s of the whole job (algorithmic
-4*d FLOPs per (query, visible key) pair) over the device-timed steps, max over ranks. Inputs are
-resident in HBM; L2 is flushed (a 256 MiB write) between timed steps, outside the timed events.
-`--impl reference` times the CPU oracle instead (bounded samples of the same workload).
+Prints ONE JSON line (rank 0). The default workload is the chunked-prefill shape (B4, 32 query /
+8 KV heads, d128, 512-query chunk over a 131072-token INT2 cache), the largest of the five.
+`value` is attention TFLOP/s of the whole job (algorithmic 4*d FLOPs per (query, visible key)
+pair) over the device-timed steps, max over ranks. Inputs are resident in HBM; L2 is flushed (a
+256 MiB write) between timed steps, outside the timed events. The `configs` block gives the same
+figures for the other workloads (attention and whole-cache quantise-append of each), `decode` the
+few-query-rows regime, `fidelity` the attention-fidelity diagnostics with and without the
+correction at INT2 and INT4. `--impl reference` times the CPU oracle instead (bounded samples of
+the same workload).
 """
 from __future__ import annotations
 
@@ -30,7 +35,9 @@ from quantized_kv_cache_19_b200 import api  # noqa: E402
 from quantized_kv_cache_19_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "corrected INT2-KV attention TFLOP/s & packed-cache GB/s, % of B200 roofline"
-DEFAULT_WORKLOAD = "bf16_int2"
+DEFAULT_WORKLOAD = "prefill_gqa"
+# the other workloads of the bench's `configs` block (tiny_f32 is a correctness-only case)
+CONFIG_WORKLOADS = ("bf16_int4", "bf16_int2", "video_dit", "long_video")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
 
@@ -144,7 +151,7 @@ class ClockSampler:
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self._stop = threading.Event()
         self._period = period_s
@@ -186,45 +193,137 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------ CPU oracle
-def oracle_sample(w, x_cpu, budget_s: float, seed: int = 0):
-    """Oracle on a bounded sample of one step: quantise the whole current chunk, then corrected
-    attention of n query rows per KV head over the full cache. Returns (seconds, flops, sample text)."""
-    import oracle
-    from threadpoolctl import threadpool_info
-    scale = 1.0 / math.sqrt(w.d)
-    K = {k: v.float().numpy() for k, v in x_cpu.items()}
-    t0 = time.perf_counter()
-    oracle.build_cache(K["K_cur"], K["V_cur"], w.bits, w.group, w.meta)      # the step's append
-    t_quant = time.perf_counter() - t0
-    cache = oracle.build_cache(K["K_src"], K["V_src"], w.bits, w.group, w.meta)   # state, untimed
-    rng = np.random.default_rng(seed)
-    total_rows = (w.Hq // w.Hkv) * w.Lq
-    order = rng.permutation(total_rows)            # rows drawn without replacement, in batches
-    n, start = 16, 0
-    spent, rows_done = 0.0, 0
-    while start < total_rows:
-        rows = np.sort(order[start:start + n])
+class OracleSample:
+    """The oracle on a bounded sample of one step: the quantise-append of the whole current chunk,
+    then corrected attention of sampled query rows of sampled (batch, KV head) pairs over their full
+    cache. The sampled heads' caches are built once, outside the timing (they are the state the
+    step starts from); the time of the whole step is extrapolated linearly in (query row, KV head)
+    pairs."""
+
+    def __init__(self, w, x_cpu, n_heads: int = 2):
+        import oracle
+        self.oracle, self.w = oracle, w
+        K = {k: v.float().numpy() for k, v in x_cpu.items()}
+        pairs = [(0, 0), (w.B - 1, w.Hkv - 1)]
+        pairs = list(dict.fromkeys(pairs))[:n_heads]
+        r = w.Hq // w.Hkv
+        self.heads = []
+        for b, h in pairs:
+            sub = {"Q": K["Q"][b:b + 1, h * r:(h + 1) * r], "K_cur": K["K_cur"][b:b + 1, h:h + 1],
+                   "V_cur": K["V_cur"][b:b + 1, h:h + 1]}
+            cache = oracle.build_cache(K["K_src"][b:b + 1, h:h + 1], K["V_src"][b:b + 1, h:h + 1],
+                                       w.bits, w.group, w.meta) if w.Lc else None
+            self.heads.append((sub, cache))
+        self.K_cur, self.V_cur = K["K_cur"], K["V_cur"]
+
+    def time(self, budget_s: float, seed: int = 0):
+        """Returns (seconds extrapolated to the whole step, flops of the step, sample text, cores)."""
+        from threadpoolctl import threadpool_info
+        w, oracle = self.w, self.oracle
+        scale = 1.0 / math.sqrt(w.d)
         t0 = time.perf_counter()
-        oracle.corrected_attention(K["Q"], cache, K["K_cur"], K["V_cur"], correct=1, causal=w.causal,
-                                   scale=scale, rows=rows)
-        spent += time.perf_counter() - t0
-        rows_done += len(rows) * w.B * w.Hkv
-        start += len(rows)
-        if spent >= budget_s:
-            break
-        n *= 2
-    blas = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
-    cores = blas or os.cpu_count()
-    all_rows = total_rows * w.B * w.Hkv
-    est_s = t_quant + spent * all_rows / rows_done           # linear in query rows
-    full_flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
-    text = (f"oracle (numpy fp64 attention, fp32 quantiser): quantise-append of the whole {w.Lcur}-token "
-            f"chunk ({t_quant:.2f} s) + corrected attention of {rows_done} of {all_rows} query rows "
-            f"({spent:.2f} s); full step extrapolated linearly in rows to {est_s:.1f} s")
-    return est_s, full_flops, text, cores
+        oracle.build_cache(self.K_cur, self.V_cur, w.bits, w.group, w.meta)      # the step's append
+        t_quant = time.perf_counter() - t0
+        rng = np.random.default_rng(seed)
+        total_rows = (w.Hq // w.Hkv) * w.Lq
+        spent, pairs_done = 0.0, 0
+        for sub, cache in self.heads:
+            order = rng.permutation(total_rows)        # rows drawn without replacement, in batches
+            n, start, head_spent = 8, 0, 0.0
+            while start < total_rows and head_spent < budget_s / len(self.heads):
+                rows = np.sort(order[start:start + n])
+                t0 = time.perf_counter()
+                oracle.corrected_attention(sub["Q"], cache, sub["K_cur"], sub["V_cur"], correct=1,
+                                           causal=w.causal, scale=scale, rows=rows)
+                head_spent += time.perf_counter() - t0
+                pairs_done += len(rows)
+                start += len(rows)
+                n *= 2
+            spent += head_spent
+        blas = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
+        cores = blas or os.cpu_count()
+        all_pairs = total_rows * w.B * w.Hkv
+        est_s = t_quant + spent * all_pairs / pairs_done           # linear in (query row, KV head) pairs
+        full_flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
+        text = (f"oracle (numpy fp64 attention, fp32 quantiser): quantise-append of the whole {w.Lcur}-token "
+                f"chunk ({t_quant:.2f} s) + corrected attention of {pairs_done} of {all_pairs} (query row, "
+                f"KV head) pairs, rows drawn at random in {len(self.heads)} KV head(s) ({spent:.2f} s); "
+                f"full step extrapolated linearly in those pairs to {est_s:.1f} s")
+        return est_s, full_flops, text, cores
 
 
 # ------------------------------------------------------------------------------------ GPU arm
+def timed_ms(fn, stream, flush, steps: int, warmup: int = 3) -> float:
+    """Mean CUDA-event time (ms) of fn() on `stream` over `steps` launches after `warmup`, with L2
+    flushed (a 256 MiB write) before every launch, outside the events."""
+    ts = []
+    for i in range(steps + warmup):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            ts.append(a.elapsed_time(b))
+    return statistics.mean(ts)
+
+
+def qa_row_bytes(w) -> int:
+    """Algorithmic HBM bytes of quantise-append per (token, KV head): read K and V, write both rows
+    of codes and both rows of (step, zero-point)."""
+    esz = 4 if w.dtype == "f32" else 2
+    return 2 * w.d * esz + 2 * (w.d * w.bits // 8) + 2 * w.n_groups * 2 * (2 if w.meta == "f16" else 4)
+
+
+def workload_figures(w, dev, peaks, flush, steps: int = 10):
+    """One workload's attention (correct=1) and quantise-append, each timed alone: attention TFLOP/s
+    against the measured bf16 peak and its packed-cache GB/s; the whole-cache quantise-append (every
+    previous chunk in one call) and the append of one chunk against measured HBM."""
+    x = make_inputs(w, device=dev)
+    cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc + w.Lcur), w.meta,
+                        device=dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm, peak_t = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+
+    def build():
+        cache.length = 0
+        api.kv_quantize_append(cache, x["K_src"], x["V_src"])
+
+    def chunk():
+        cache.length = w.Lc
+        api.kv_quantize_append(cache, x["K_cur"], x["V_cur"])
+
+    full_ms = timed_ms(build, stream, flush, steps)
+    chunk_ms = timed_ms(chunk, stream, flush, steps)
+    cache.length = w.Lc
+    O = torch.empty_like(x["Q"])
+    LSE = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
+    attn_ms = timed_ms(lambda: api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1,
+                                                       causal=w.causal, out=O, lse=LSE), stream, flush, steps)
+    if api.device_status() != 0:
+        raise RuntimeError(f"device status after the {w.name} figures")
+    flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
+    tf = flops / (attn_ms * 1e-3) / 1e12
+    full_bytes = w.B * w.Hkv * w.Lc * qa_row_bytes(w)
+    chunk_bytes = w.B * w.Hkv * w.Lcur * qa_row_bytes(w)
+    out = {"workload": describe(w),
+           "attention": {"kernel": "corrected_attention_kernel", "bound": "tensor",
+                         "ms_per_launch": round(attn_ms, 5), "flops_per_launch": flops,
+                         "achieved_tflops": round(tf, 2), "peak_tflops": peak_t, "frac": round(tf / peak_t, 4),
+                         "packed_cache_gbs": round(cache.packed_bytes(w.Lc) / (attn_ms * 1e-3) / 1e9, 1)},
+           "quant_append_full_cache": {"kernel": "quantize_append_kernel", "bound": "hbm", "tokens": w.Lc,
+                                       "ms_per_launch": round(full_ms, 5), "bytes_per_launch": full_bytes,
+                                       "achieved_gbs": round(full_bytes / (full_ms * 1e-3) / 1e9, 1),
+                                       "peak_gbs": hbm, "frac": round(full_bytes / (full_ms * 1e-3) / 1e9 / hbm, 4)},
+           "quant_append_chunk": {"tokens": w.Lcur, "ms_per_launch": round(chunk_ms, 5),
+                                  "bytes_per_launch": chunk_bytes,
+                                  "achieved_gbs": round(chunk_bytes / (chunk_ms * 1e-3) / 1e9, 1)}}
+    del x, cache, O, LSE
+    torch.cuda.empty_cache()
+    return out
+
+
 def decode_sweep(dev, peaks, flush, steps: int = 20):
     """Few query rows per KV head over the chunked-prefill workload's 131072-token INT2 cache
     (B4, 32 query / 8 KV heads): the regime where attention reads the packed cache once and the
@@ -233,9 +332,7 @@ def decode_sweep(dev, peaks, flush, steps: int = 20):
     x = make_inputs(base.with_(Lq=16, Lcur=16), device=dev)
     cache = api.KVCache(base.B, base.Hkv, base.d, base.bits, base.group, api.round_capacity(base.Lc),
                         base.meta, device=dev)
-    for t0 in range(0, base.Lc, 16384):
-        api.kv_quantize_append(cache, x["K_src"][:, :, t0:t0 + 16384].contiguous(),
-                               x["V_src"][:, :, t0:t0 + 16384].contiguous())
+    api.kv_quantize_append(cache, x["K_src"], x["V_src"])
     stream = torch.cuda.current_stream(dev)
     out = {"workload": "prefill_gqa cache (B4 Hq32 Hkv8 d128 Lc131072 INT2 G64 f32 meta), Lcur = Lq, causal",
            "bound": "hbm", "peak_gbs": float(peaks["hbm_gbs"]), "points": []}
@@ -247,17 +344,8 @@ def decode_sweep(dev, peaks, flush, steps: int = 20):
         L = torch.empty(base.B, base.Hq, Lq, dtype=torch.float32, device=dev)
         nws = api.attention_workspace_bytes(cache, base.Hq, Lq, Lq)
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
-        ts = []
-        for i in range(steps + 3):
-            flush.fill_(i & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            api.corrected_attention(Q, cache, Kc, Vc, correct=1, causal=True, out=O, lse=L, workspace=ws)
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(a.elapsed_time(b))
-        ms = statistics.mean(ts)
+        ms = timed_ms(lambda: api.corrected_attention(Q, cache, Kc, Vc, correct=1, causal=True, out=O, lse=L,
+                                                      workspace=ws), stream, flush, steps)
         gbs = cache.packed_bytes(base.Lc) / (ms * 1e-3) / 1e9
         out["points"].append({"Lq": Lq, "rows_per_kv_head": 4 * Lq, "ms": round(ms, 4),
                               "workspace_bytes": nws, "packed_cache_gbs": round(gbs, 1),
@@ -269,51 +357,61 @@ def decode_sweep(dev, peaks, flush, steps: int = 20):
     return out
 
 
-def fidelity_leg(w, x, cache, dev, flush, steps: int = 10):
-    """Attention-fidelity diagnostics (cached mass, KL, top-1 agreement, top-5 recall) over the
-    bench workload, correct=1, top lists written. fp32 CUDA-core arithmetic: 4d FLOP per (query row,
-    cached key) pair (two dot products) and 2d per visible current key, against the fp32 FMA peak
-    148 SMs x 128 lanes x 2 FLOP x the maximum SM clock."""
+def fidelity_means(st) -> dict:
+    return {"mass_ref": round(st[..., 2].mean().item(), 5), "mass_q": round(st[..., 3].mean().item(), 5),
+            "kl": round(st[..., 4].mean().item(), 5), "token_drift": round(1.0 - st[..., 5].mean().item(), 5),
+            "top5_recall": round(st[..., 6].mean().item(), 5)}
+
+
+def fidelity_leg(dev, flush, steps: int = 10):
+    """Attention-fidelity diagnostics (cached mass under the reference and the quantised softmax,
+    KL(P_ref || P_q), token drift, top-5 recall), row means, without (correct=0) and with (correct=1)
+    the correction, at INT2 and INT4, on the bf16 workload and on the video-DiT workload. The kernel
+    (fp32 CUDA cores) is timed on bf16_int2 with correct=1 and top lists written: 4d FLOP per (query
+    row, cached key) pair (two dot products) and 2d per visible current key, against the fp32 FMA
+    peak 148 SMs x 128 lanes x 2 FLOP x the maximum SM clock."""
     props = torch.cuda.get_device_properties(dev)
     sm_mhz = float(load_peaks()[0].get("sm_max_mhz", 1965.0))
     peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
-    rows = w.B * w.Hq * w.Lq
-    if w.causal:
-        vis_cur = sum(max(0, min(w.Lcur, i + (w.Lcur - w.Lq) + 1)) for i in range(w.Lq)) * w.B * w.Hq
-    else:
-        vis_cur = rows * w.Lcur
-    flops = 4 * w.d * rows * w.Lc + 2 * w.d * vis_cur
     stream = torch.cuda.current_stream(dev)
-    cache.length = w.Lc                      # the cache holds the quantised K_src in positions [0, Lc)
-    ts = []
-    for i in range(steps + 3):
-        flush.fill_(i & 0xFF)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        st, top = api.attention_fidelity(x["Q"], cache, x["K_src"], x["K_cur"], correct=1, causal=w.causal)
-        b.record(stream)
-        torch.cuda.synchronize()
-        if i >= 3:
-            ts.append(a.elapsed_time(b))
+    out = {"kernel": "attention_fidelity_kernel", "compared": []}
+    cases = [("bf16_int2", WORKLOADS["bf16_int2"]), ("bf16_int4", WORKLOADS["bf16_int4"]),
+             ("video_dit", WORKLOADS["video_dit"]), ("video_dit at INT4", WORKLOADS["video_dit"].with_(bits=4))]
+    for label, w in cases:
+        x = make_inputs(w, device=dev)
+        cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc), w.meta, device=dev)
+        api.kv_quantize_append(cache, x["K_src"], x["V_src"])
+        rec = {"workload": label, "bits": w.bits, "group": w.group}
+        for correct in (0, 1):
+            st, _ = api.attention_fidelity(x["Q"], cache, x["K_src"], x["K_cur"], correct=correct, causal=w.causal)
+            rec[f"correct{correct}"] = fidelity_means(st)
+        out["compared"].append(rec)
+        if label == "bf16_int2":
+            rows = w.B * w.Hq * w.Lq
+            vis_cur = rows * w.Lcur
+            flops = 4 * w.d * rows * w.Lc + 2 * w.d * vis_cur
+            ms = timed_ms(lambda: api.attention_fidelity(x["Q"], cache, x["K_src"], x["K_cur"], correct=1,
+                                                         causal=w.causal), stream, flush, steps)
+            tf = flops / (ms * 1e-3) / 1e12
+            out.update({"timed_on": "bf16_int2, correct=1, top lists written", "bound": "alu",
+                        "ms_per_launch": round(ms, 4), "flops_per_launch": flops, "achieved": round(tf, 2),
+                        "peak": round(peak, 1), "unit": "TFLOP/s",
+                        "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x max SM clock", "frac": round(tf / peak, 4),
+                        "traffic": ncu_traffic("attention_fidelity_kernel", w.name)})
+        del x, cache
+        torch.cuda.empty_cache()
     if api.device_status() != 0:
         raise RuntimeError("device status after the fidelity diagnostics")
-    ms = statistics.mean(ts)
-    tf = flops / (ms * 1e-3) / 1e12
-    return {"kernel": "attention_fidelity_kernel", "bound": "alu", "ms_per_launch": round(ms, 4),
-            "flops_per_launch": flops, "achieved": round(tf, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-            "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x max SM clock", "frac": round(tf / peak, 4),
-            "traffic": ncu_traffic("attention_fidelity_kernel", w.name),
-            "means": {"mass_ref": round(st[..., 2].mean().item(), 5), "mass_q": round(st[..., 3].mean().item(), 5),
-                      "kl": round(st[..., 4].mean().item(), 5),
-                      "token_drift": round(1.0 - st[..., 5].mean().item(), 5),
-                      "top5_recall": round(st[..., 6].mean().item(), 5)}}
+    return out
 
 
-def key_channel_leg(w, x, dev, flush, T: int = 32, steps: int = 10):
-    """Per-channel keys along tokens (blocks of T positions, KIVI's group size of 32) on the bench
-    workload: the whole-cache quantise-append (keys per channel, values per token; HBM-bound) and
+def key_channel_leg(dev, flush, T: int = 32, steps: int = 10):
+    """Per-channel keys along tokens (blocks of T positions, KIVI's group size of 32) on the bf16
+    INT2 workload: the whole-cache quantise-append (keys per channel, values per token; HBM-bound) and
     corrected attention (correct=1) on the fp32 CUDA-core kernel that serves this layout, against
     the fp32 FMA peak."""
+    w = WORKLOADS["bf16_int2"]
+    x = make_inputs(w, device=dev)
     props = torch.cuda.get_device_properties(dev)
     sm_mhz = float(load_peaks()[0].get("sm_max_mhz", 1965.0))
     fp32_peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
@@ -322,37 +420,25 @@ def key_channel_leg(w, x, dev, flush, T: int = 32, steps: int = 10):
                         key_block=T)
     stream = torch.cuda.current_stream(dev)
 
-    def timed(fn):
-        ts = []
-        for i in range(steps + 3):
-            flush.fill_(i & 0xFF)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(a.elapsed_time(b))
-        return statistics.mean(ts)
-
     def quant():
         cache.length = 0
         api.kv_quantize_append(cache, x["K_src"], x["V_src"])
 
-    q_ms = timed(quant)
+    q_ms = timed_ms(quant, stream, flush, steps)
     in_bytes = x["K_src"].element_size()
     q_bytes = 2 * w.B * w.Hkv * w.Lc * w.d * in_bytes + cache.packed_bytes(w.Lc)
     O = torch.empty_like(x["Q"])
     LSE = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
-    a_ms = timed(lambda: api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1,
-                                                 causal=w.causal, out=O, lse=LSE))
+    a_ms = timed_ms(lambda: api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1,
+                                                    causal=w.causal, out=O, lse=LSE), stream, flush, steps)
     if api.device_status() != 0:
         raise RuntimeError("device status after the per-channel key leg")
     flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
     tf = flops / (a_ms * 1e-3) / 1e12
     gbs = q_bytes / (q_ms * 1e-3) / 1e9
-    del cache
-    return {"key_block": T,
+    del cache, x
+    torch.cuda.empty_cache()
+    return {"workload": describe(w), "key_block": T,
             "quantize_append_full_cache": {"bound": "hbm", "ms": round(q_ms, 4), "bytes": q_bytes,
                                            "achieved_gbs": round(gbs, 1), "peak_gbs": hbm,
                                            "frac": round(gbs / hbm, 4)},
@@ -361,6 +447,73 @@ def key_channel_leg(w, x, dev, flush, T: int = 32, steps: int = 10):
                           "achieved": round(tf, 2), "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
                           "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x max SM clock",
                           "frac": round(tf / fp32_peak, 4)}}
+
+
+def e2e_leg(w, x, cache, dev, flush, n_steps: int):
+    """The step through the public API with host buffers: every step uploads its Q, K_cur and V_cur
+    from pinned host memory and reads O and LSE back into pinned host memory. Uploads and read-backs
+    run on two copy streams with two sets of device buffers, so that step i+1's upload and step
+    i-1's read-back overlap step i's kernels, as a serving loop would run it. Returns (ms per step,
+    H2D bytes per step, D2H bytes per step); the time runs from the first upload to the last
+    read-back, on the device."""
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    names = ("Q", "K_cur", "V_cur")
+    pin = [{k: x[k].cpu().pin_memory() for k in names} for _ in range(2)]
+    d_in = [{k: torch.empty_like(x[k]) for k in names} for _ in range(2)]
+    d_o = [torch.empty_like(x["Q"]) for _ in range(2)]
+    d_l = [torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev) for _ in range(2)]
+    h_o = [torch.empty(d_o[0].shape, dtype=d_o[0].dtype).pin_memory() for _ in range(2)]
+    h_l = [torch.empty(d_l[0].shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
+
+    def upload(i):
+        s = i % 2
+        with torch.cuda.stream(up):
+            if used[s]:
+                up.wait_event(computed[s])         # step i-2 has finished reading these inputs
+            for k in names:
+                d_in[s][k].copy_(pin[s][k], non_blocking=True)
+            uploaded[s].record(up)
+
+    def run(n, timed):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if timed:
+            start.record(up)
+        upload(0)
+        for i in range(n):
+            s = i % 2
+            if i + 1 < n:
+                upload(i + 1)
+            comp.wait_event(uploaded[s])
+            if used[s]:
+                comp.wait_event(read[s])             # step i-2's outputs have been read back
+            cache.length = w.Lc
+            api.corrected_attention(d_in[s]["Q"], cache, d_in[s]["K_cur"], d_in[s]["V_cur"], correct=1,
+                                    causal=w.causal, out=d_o[s], lse=d_l[s])
+            api.kv_quantize_append(cache, d_in[s]["K_cur"], d_in[s]["V_cur"])
+            computed[s].record(comp)
+            used[s] = True
+            with torch.cuda.stream(down):
+                down.wait_event(computed[s])
+                h_o[s].copy_(d_o[s], non_blocking=True)
+                h_l[s].copy_(d_l[s], non_blocking=True)
+                read[s].record(down)
+        if timed:
+            end.record(down)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / n if timed else 0.0
+
+    flush.fill_(0)
+    run(3, False)
+    torch.cuda.synchronize()
+    ms = run(n_steps, True)
+    h2d = sum(t.numel() * t.element_size() for t in pin[0].values())
+    d2h = d_o[0].numel() * d_o[0].element_size() + d_l[0].numel() * 4
+    return ms, h2d, d2h
 
 
 def run_ours(args, world, rank, local):
@@ -380,6 +533,8 @@ def run_ours(args, world, rank, local):
     LSE = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    ws_bytes = api.attention_workspace_bytes(cache, w.Hq, w.Lq, w.Lcur)
+    launches_per_step = 2 + (1 if ws_bytes else 0)            # attention (+ merge of a key split) + append
 
     def step():
         cache.length = w.Lc
@@ -415,44 +570,15 @@ def run_ours(args, world, rank, local):
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
 
-    # end to end through the public API with host buffers: H2D of the step's inputs, D2H of O, LSE
-    pin = {k: x[k].cpu().pin_memory() for k in ("Q", "K_cur", "V_cur")}
-    dev_in = {k: torch.empty_like(x[k]) for k in pin}
-    O_host = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-    L_host = torch.empty(LSE.shape, dtype=LSE.dtype).pin_memory()
-    n_e2e = min(K, 50)
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_e2e)]
-    for i in range(n_e2e + 3):
-        flush.fill_(i & 0xFF)
-        if i >= 3:
-            e2e_ev[i - 3][0].record(stream)
-        for k in pin:
-            dev_in[k].copy_(pin[k], non_blocking=True)
-        cache.length = w.Lc
-        api.corrected_attention(dev_in["Q"], cache, dev_in["K_cur"], dev_in["V_cur"], correct=1,
-                                causal=w.causal, out=O, lse=LSE)
-        api.kv_quantize_append(cache, dev_in["K_cur"], dev_in["V_cur"])
-        O_host.copy_(O, non_blocking=True)
-        L_host.copy_(LSE, non_blocking=True)
-        if i >= 3:
-            e2e_ev[i - 3][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in e2e_ev)
+    # end to end through the public API with host buffers (pipelined uploads and read-backs)
+    e2e_ms, h2d_bytes, d2h_bytes = e2e_leg(w, x, cache, dev, flush, min(K, 50))
 
     # whole-cache build: every previous chunk quantised in one call (the HBM-bound figure of the
-    # quantiser; a single 1024-token chunk is too small to leave launch latency behind)
-    n_full = 20
-    full_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_full)]
-    for i in range(n_full + 3):
-        flush.fill_(i & 0xFF)
+    # quantiser; a single chunk is too small to leave launch latency behind)
+    def build():
         cache.length = 0
-        if i >= 3:
-            full_ev[i - 3][0].record(stream)
         api.kv_quantize_append(cache, x["K_src"], x["V_src"])
-        if i >= 3:
-            full_ev[i - 3][1].record(stream)
-    torch.cuda.synchronize()
-    full_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in full_ev)
+    full_ms = timed_ms(build, stream, flush, 20)
     cache.length = w.Lc
 
     flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
@@ -463,12 +589,14 @@ def run_ours(args, world, rank, local):
     ms_attn = reduce_max(mean_attn, world, dev)
     ms_e2e = reduce_max(e2e_ms, world, dev)
     packed = cache.packed_bytes(w.Lc)
-    esz = x["K_cur"].element_size()
-    row_bytes = 2 * w.d * esz + 2 * (w.d * w.bits // 8) + 2 * w.n_groups * 2 * (2 if w.meta == "f16" else 4)
-    qa_bytes = w.B * w.Hkv * w.Lcur * row_bytes
-    full_bytes = w.B * w.Hkv * w.Lc * row_bytes
+    qa_bytes = w.B * w.Hkv * w.Lcur * qa_row_bytes(w)
+    full_bytes = w.B * w.Hkv * w.Lc * qa_row_bytes(w)
     peak_t = float(peaks["bf16_tflops"])
     achieved = flops / (ms_attn * 1e-3) / 1e12
+    clk = clocks.summary()
+    if clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        # the attention time the kernel would take at the maximum SM clock, if it scaled with it
+        clk["attention_ms_at_max_clock"] = round(ms_attn * clk["sm_mhz"] / clk["sm_max_mhz"], 5)
     result = {
         "metric": METRIC,
         "value": round(world * flops / (ms_step * 1e-3) / 1e12, 3),
@@ -500,21 +628,25 @@ def run_ours(args, world, rank, local):
                                         "frac": round(full_bytes / (full_ms * 1e-3) / 1e9 /
                                                       float(peaks["hbm_gbs"]), 4)}},
         "e2e": {"value": round(world * flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-                "ms_per_step": round(ms_e2e, 5),
-                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
-                "d2h_bytes_per_step": O.numel() * O.element_size() + LSE.numel() * LSE.element_size()},
-        "gpu_launches": 2 * K,
-        "clocks": clocks.summary(),
+                "ms_per_step": round(ms_e2e, 5), "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+                "how": "pinned host buffers; uploads and read-backs on two copy streams, double-buffered"},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clk,
     }
+    del x, cache, O, LSE
+    torch.cuda.empty_cache()
+    if not args.no_configs:
+        result["configs"] = [workload_figures(WORKLOADS[n], dev, peaks, flush) for n in CONFIG_WORKLOADS
+                             if n != w.name]
     if not args.no_fidelity:
-        result["fidelity"] = fidelity_leg(w, x, cache, dev, flush)
+        result["fidelity"] = fidelity_leg(dev, flush)
     if not args.no_key_channel:
-        result["key_per_channel"] = key_channel_leg(w, x, dev, flush)
+        result["key_per_channel"] = key_channel_leg(dev, flush)
     if not args.no_decode:
         result["decode"] = decode_sweep(dev, peaks, flush)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         x_cpu = make_inputs(w, device="cpu")
-        est_s, full_flops, text, cores = oracle_sample(w, x_cpu, args.cpu_budget)
+        est_s, full_flops, text, cores = OracleSample(w, x_cpu).time(args.cpu_budget)
         result["cpu_baseline"] = {"value": round(full_flops / est_s / 1e12, 6), "unit": "TFLOP/s",
                                   "cores": cores, "kind": "oracle", "sample": text}
     return result
@@ -526,10 +658,11 @@ def run_reference(args, world, rank):
         return None
     w = WORKLOADS[args.workload]
     x_cpu = make_inputs(w, device="cpu")
-    per_step = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    sample = OracleSample(w, x_cpu)
+    per_step = max(0.5, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     times, text, cores = [], "", os.cpu_count()
     for i in range(args.warmup + args.steps):
-        est_s, full_flops, text, cores = oracle_sample(w, x_cpu, per_step, seed=i)
+        est_s, full_flops, text, cores = sample.time(per_step, seed=i)
         if i >= args.warmup:
             times.append(est_s)
     mean_s = statistics.mean(times)
@@ -547,7 +680,7 @@ def run_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -556,6 +689,7 @@ def main(argv=None):
     ap.add_argument("--no-decode", action="store_true", help="skip the few-query-rows (decode) sweep")
     ap.add_argument("--no-fidelity", action="store_true", help="skip the attention-fidelity diagnostics")
     ap.add_argument("--no-key-channel", action="store_true", help="skip the per-channel key layout leg")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' figures")
     ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
                     help="store the DRAM bytes per launch of an ncu report (taken on --workload) and exit")
     ap.add_argument("--record-command", default="", help="the command line that made the report")

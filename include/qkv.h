@@ -163,10 +163,13 @@ qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_
  * results go to a scratch array that the library itself holds in device memory, 8 MiB on every GPU
  * that loads the library, kept until the process exits. No call allocates or frees memory.
  *  - A shape whose split needs more than 8 MiB of scratch (corrected_attention_workspace_bytes()
- *    larger than 8 MiB) is rejected with QKV_ERR_UNSUPPORTED; corrected_attention with a workspace
- *    handles it. Caches with per-channel keys (key_block > 0) run unsplit here and need no scratch.
+ *    larger than 8 MiB) splits its cached keys fewer ways, as many as the 8 MiB hold the partials
+ *    of, or runs unsplit when fewer than two fit: the results are the same, only the number of
+ *    CTAs that share the cache reads differs. Caches with per-channel keys (key_block > 0) run
+ *    unsplit here and need no scratch.
  *  - The first call on a device that needs the scratch looks up the array's device address (with
- *    that device current); make that first call before any stream capture.
+ *    that device current), and looks it up again after the device's context has been re-created
+ *    (e.g. after cudaDeviceReset); make that first call before any stream capture.
  *  - All calls share the one array: every value a call reads from it was written by the same call,
  *    but two calls that overlap on the GPU (different streams, or different host threads) race on
  *    it and must be serialised by the caller.
@@ -212,6 +215,16 @@ qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q, int64_t
                               const qkv_cache* cache, const void* K_ref, const void* K_cur,
                               int64_t L_cur, int32_t correct, int32_t causal_cur, float scale,
                               float* stats, int32_t* top, void* stream);
+
+/*
+ * Bound of every internal wait of the kernels launched from now on by this process, in SM clock
+ * cycles (default 2e9, about a second; 0 restores the default); *previous (if not NULL) receives
+ * the bound in force before. For tests of the timeout path: with a bound of a few cycles the
+ * attention kernel's waits give up at once, the kernel returns early with its outputs undefined,
+ * and qkv_device_status() reports QKV_ERR_TIMEOUT. The waits on the way out of a kernel (for its
+ * own copies and tensor-core operations in flight) keep the default bound. Host only.
+ */
+qkv_status qkv_set_wait_limit(int64_t cycles, int64_t* previous);
 
 /*
  * Reads the library's device status word (0 = no error, else a qkv_status such as

@@ -70,6 +70,7 @@ _SIGS = {
                                           ctypes.POINTER(QkvCacheDesc), _P, _P, ctypes.c_int64,
                                           ctypes.c_int32, ctypes.c_int32, ctypes.c_float, _P, _P, _P]),
     "qkv_device_status": (ctypes.c_int, [ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
+    "qkv_set_wait_limit": (ctypes.c_int, [ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]),
 }
 
 
@@ -309,6 +310,15 @@ def device_status(reset: bool = True) -> int:
     code = ctypes.c_int32()
     _check(lib.qkv_device_status(int(reset), ctypes.byref(code)))
     return int(code.value)
+
+
+def set_wait_limit(cycles: int) -> int:
+    """Bound, in SM clock cycles, of the internal waits of kernels launched from now on (0 restores
+    the default of 2e9); returns the previous bound. For tests of the timeout path."""
+    lib = load_library()
+    prev = ctypes.c_int64()
+    _check(lib.qkv_set_wait_limit(int(cycles), ctypes.byref(prev)))
+    return int(prev.value)
 
 
 def attention_flops(B: int, Hq: int, Lq: int, Lc: int, Lcur: int, d: int, causal: bool = False) -> float:

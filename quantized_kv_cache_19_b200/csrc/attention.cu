@@ -460,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       // O += P_i V_i once the softmax wrote P_i and V_i is in smem.
       auto issue_pv = [&](int i) -> bool {
         const int vb = i & 1, pb = i % C::kPB;
-        if (!mbar_wait(bar(B_P_FULL + pb), (i / C::kPB) & 1, abort_flag, p.status)) return false;
-        if (!mbar_wait(bar(B_VH_FULL + vb), (i >> 1) & 1, abort_flag, p.status)) return false;
+        if (!mbar_wait(bar(B_P_FULL + pb), (i / C::kPB) & 1, abort_flag, p.status, p.wait_limit)) return false;
+        if (!mbar_wait(bar(B_VH_FULL + vb), (i >> 1) & 1, abort_flag, p.status, p.wait_limit)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < N / 16; ++kk)   // 16 keys = two 1024-byte atoms per step
@@ -471,14 +471,14 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         tc_commit(bar(B_PV_DONE + pb));
         return true;
       };
-      bool ok = T > 0 && mbar_wait(bar(B_Q_FULL), 0, abort_flag, p.status);
+      bool ok = T > 0 && mbar_wait(bar(B_Q_FULL), 0, abort_flag, p.status, p.wait_limit);
       if (ok) tc_fence_after();
       // In order: S_j (once K_j is in smem and its S buffer was read by the softmax), then
       // P_{j-1}.V_{j-1}.
       for (int j = 0; j < T && ok; ++j) {
         const int kb = j & 1, sb = j % C::kSB;
-        if (!mbar_wait(bar(B_KH_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        if (j >= C::kSB && !mbar_wait(bar(B_S_FREE + sb), ((j - C::kSB) / C::kSB) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (!mbar_wait(bar(B_KH_FULL + kb), (j >> 1) & 1, abort_flag, p.status, p.wait_limit)) { ok = false; break; }
+        if (j >= C::kSB && !mbar_wait(bar(B_S_FREE + sb), ((j - C::kSB) / C::kSB) & 1, abort_flag, p.status, p.wait_limit)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tm_sj = tm_s + sb * C::kSCols;
         // K tile [d/64][N keys][64], 128B swizzle, K-major: 16 channels per step (32 bytes inside
@@ -515,13 +515,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* kt = smem + L.kt + sb * C::kTile;
-      if (!warp_wait(bar(B_KH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+      if (!warp_wait(bar(B_KH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status, p.wait_limit)) break;
       if (j < Tc) {
         const int s = j % kStages, k = j / kStages;
         const int64_t rem = p.Lc - static_cast<int64_t>(c0 + j) * N;
         const int valid = static_cast<int>(rem < N ? rem : N);
         const uint8_t* kcodes = smem + L.pk + s * L.stage;
-        if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
+        if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status, p.wait_limit)) break;
         using CodeVec = typename CodeVecT<BITS>::type;
         // One item per iteration with the next item's codes already loaded (shared-memory loads
         // take ~170 cycles while the tensor core reads its operands), the loop itself not
@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         }
         // Per-key constants of the tile: scales a for the softmax (once it has read the previous
         // ones from this buffer) and the key extras of the S MMA.
-        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status, p.wait_limit)) break;
         const uint8_t* kmeta = kcodes + C::kCodes;
         float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
         constexpr int kItersC = (N * NG + kKThreads - 1) / kKThreads;
@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         fence_async_smem();
         // Scales of the current tile: the plain score scale for every key and group, so that the
         // softmax forms every tile's scores the same way.
-        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+        if (!warp_wait(bar(B_KC_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status, p.wait_limit)) break;
         float* kc = reinterpret_cast<float*>(kconst + sb * (C::kKconst / 16));
 #pragma unroll 1
         for (int e = t; e < static_cast<int>(C::kKconst / 4); e += kKThreads) {
@@ -622,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     int next_load = 0;
     auto issue_load = [&]() -> bool {
       const int s = next_load % kStages, k = next_load / kStages;
-      if (!mbar_wait(bar(B_PK_EMPTY + s), (k & 1) ^ 1, abort_flag, p.status)) return false;
+      if (!mbar_wait(bar(B_PK_EMPTY + s), (k & 1) ^ 1, abort_flag, p.status, p.wait_limit)) return false;
       const uint32_t dst = smem_u32(smem + L.pk + s * L.stage);
       const int64_t row0 = static_cast<int64_t>(bh) * p.capacity + static_cast<int64_t>(c0 + next_load) * N;
       const uint32_t fb = bar(B_PK_FULL + s);
@@ -641,14 +641,14 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* vt = smem + L.vt + sb * C::kTile;
-      if (!warp_wait(bar(B_VH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status)) break;
+      if (!warp_wait(bar(B_VH_EMPTY + sb), (n & 1) ^ 1, abort_flag, p.status, p.wait_limit)) break;
       if (j < Tc) {
         const int s = j % kStages, k = j / kStages;
         const int64_t rem = p.Lc - static_cast<int64_t>(c0 + j) * N;
         const int valid = static_cast<int>(rem < N ? rem : N);
         const uint8_t* vcodes = smem + L.pk + s * L.stage + C::kCodes + L.meta;
         const uint8_t* vmeta = vcodes + C::kCodes;
-        if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status)) break;
+        if (!warp_wait(bar(B_PK_FULL + s), k & 1, abort_flag, p.status, p.wait_limit)) break;
         using CodeVec = typename CodeVecT<BITS>::type;
         // One item per iteration with the next item's codes and (step, zero-point) already loaded
         // (shared-memory loads are slow while the tensor core reads its operands); the loop itself
@@ -779,14 +779,18 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     float m_run = -INFINITY;   // max used for the exponentials so far (log2 units), same in both halves
     float l_run = 0.f;         // this half's part of the softmax denominator
     const float2 scale2 = make_float2(p.scale_log2, p.scale_log2);
+    // ok turns false when one of this warp's waits gives up. The eight softmax warps share named
+    // barrier 1, so none of them leaves the tile loop on its own: a failed warp skips its work and
+    // the warps leave together at the next row-max exchange, which ORs their failures, so that
+    // every warp executes the same sequence of barriers (one per tile, then one in the epilogue).
     bool ok = true;
     // S columns are read in chunks of kCK keys (NA * kCK registers); tcgen05.wait::ld waits for
     // every load of a chunk.
     constexpr int kCK = C::NA == 1 ? 32 : 64 / C::NA;
-    for (int j = 0; j < T && ok; ++j) {
+    for (int j = 0; j < T; ++j) {
       const int kb = j & 1, sbuf = j % C::kSB, pb = j % C::kPB;
       const bool cached = j < Tc;
-      if (!warp_wait(bar(B_S_FULL + sbuf), (j / C::kSB) & 1, abort_flag, p.status)) { ok = false; break; }
+      if (ok && !warp_wait(bar(B_S_FULL + sbuf), (j / C::kSB) & 1, abort_flag, p.status, p.wait_limit)) ok = false;
       tc_fence_after();
       const uint32_t tm_s = tmem + lane_off + kColS + sbuf * C::kSCols + kbase_h;
       float2 s2[NH / 2];         // scores of this half's key pairs (log2 units)
@@ -803,12 +807,14 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         }
         valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
       }
-      if (!warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+      if (ok && !warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status, p.wait_limit)) ok = false;
       // s = sum_g a_g * S_g: per-key group scales for cached tiles, the score scale for current ones.
       const float4* ka = kconst + kb * (C::kKconst / 16);
       const float4* kd4 = kconst + (2 + kb) * (C::kKconst / 16);
 #pragma unroll
       for (int c0 = 0; c0 < NH; c0 += kCK) {
+        // (After a failed wait these loads read whatever the accumulators hold; the values are
+        // dropped at the exchange below, where the warps leave the loop.)
         uint32_t r[C::NA][kCK];
 #pragma unroll
         for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
@@ -838,7 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
+      if (ok && lane == 0) {
         mbar_arrive(bar(B_S_FREE + sbuf));
         mbar_arrive(bar(B_KC_EMPTY + kb));
       }
@@ -860,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       }
       const float m_half = fmax3(fmaxf(m0, m1), m2, m3);
       xmax[((j & 1) * 2 + half) * kBM + row] = m_half;
-      named_sync(1, 256);
+      if (named_sync_or(1, 256, !ok)) { ok = false; break; }
       const float m_tile = fmaxf(m_half, xmax[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
       // Lazy rescaling: keep the old max unless the new one exceeds it by the threshold.
       const bool need = (m_tile > m_run + kRescaleThreshold) ||
@@ -874,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
       // O is rescaled only after the previous P.V has finished (rare with lazy rescaling).
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        if (!warp_wait(bar(B_PV_DONE + (j - 1) % C::kPB), ((j - 1) / C::kPB) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (!warp_wait(bar(B_PV_DONE + (j - 1) % C::kPB), ((j - 1) / C::kPB) & 1, abort_flag, p.status, p.wait_limit)) { ok = false; continue; }
         tc_fence_after();
         const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
         const float2 f2 = make_float2(factor, factor);
@@ -894,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       }
       // P buffer pb was last read by P_{j-kPB}.V_{j-kPB}.
       if (j >= C::kPB) {
-        if (!warp_wait(bar(B_PV_DONE + pb), ((j - C::kPB) / C::kPB) & 1, abort_flag, p.status)) { ok = false; break; }
+        if (!warp_wait(bar(B_PV_DONE + pb), ((j - C::kPB) / C::kPB) & 1, abort_flag, p.status, p.wait_limit)) { ok = false; continue; }
         tc_fence_after();
       }
       const float2 mneg = make_float2(-m_use, -m_use);
@@ -918,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     // Epilogue: combine the two halves' denominators, O / l (each half writes half the columns), LSE.
     bool have_o = false;
     if (ok && T > 0) {
-      have_o = warp_wait(bar(B_PV_DONE + (T - 1) % C::kPB), ((T - 1) / C::kPB) & 1, abort_flag, p.status);
+      have_o = warp_wait(bar(B_PV_DONE + (T - 1) % C::kPB), ((T - 1) / C::kPB) & 1, abort_flag, p.status, p.wait_limit);
       tc_fence_after();
     }
     xsum[half * kBM + row] = l_run;

@@ -4,12 +4,15 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
+#include <mutex>
 #include <string>
 
 #include "../../include/qkv.h"
 #include "channel.h"
 #include "fidelity.h"
 #include "qkv_internal.h"
+#include "symbol_cache.h"
 
 #define QKV_API extern "C" __attribute__((visibility("default")))
 
@@ -17,6 +20,9 @@ namespace qkv {
 
 // Device status word of this library: 0 = ok, else a negative qkv_status set by a kernel.
 __device__ int g_device_status;
+
+// Bound of the progress waits of kernels launched from now on, in SM clock cycles.
+static std::atomic<long long> g_wait_limit{kDefaultWaitLimitCycles};
 
 namespace {
 
@@ -39,19 +45,69 @@ qkv_status cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Address of g_device_status on the current device (looked up once per device).
-int* status_word(cudaError_t* err) {
-  static int* addr[64] = {nullptr};
+// Unique id of the current CUDA context (0 if there is none, or if the driver cannot say). The
+// driver calls are reached through the runtime's entry-point query, so the library does not link
+// the driver library itself.
+unsigned long long current_context_id() {
+  using GetCurrent = int (*)(void**);
+  using GetId = int (*)(void*, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return 0;
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != 0 || ctx == nullptr || get_id(ctx, &id) != 0) return 0;
+  return id;
+}
+
+// Device address of one of the library's __device__ variables on the current device, looked up
+// again whenever the current context is not the one the remembered address was taken in.
+template <class T>
+void* symbol_address(SymbolAddressCache& cache, const T& symbol, cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (addr[dev] == nullptr) {
+  if (*err != cudaSuccess) return nullptr;
+  unsigned long long ctx = current_context_id();
+  if (ctx == 0) {
+    // No context yet on this thread: the runtime creates the device's primary context on the
+    // first call that needs one, such as this lookup; then its id can be read.
     void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_device_status);
+    *err = cudaGetSymbolAddress(&p, symbol);
     if (*err != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<int*>(p);
+    ctx = current_context_id();
   }
-  return addr[dev];
+  void* out = nullptr;
+  cudaError_t lookup_err = cudaSuccess;
+  const int rc = cache.get(dev, ctx, [&](void** p) {
+    lookup_err = cudaGetSymbolAddress(p, symbol);
+    return lookup_err == cudaSuccess ? 0 : 1;
+  }, &out);
+  if (rc != 0) {
+    *err = rc == -1 ? cudaErrorInvalidDevice : lookup_err;
+    return nullptr;
+  }
+  *err = cudaSuccess;
+  return out;
+}
+
+SymbolAddressCache g_status_addr;
+
+// Address of g_device_status on the current device, in the current context.
+int* status_word(cudaError_t* err) {
+  return static_cast<int*>(symbol_address(g_status_addr, g_device_status, err));
 }
 
 qkv_status check_shape(int32_t B, int32_t H_kv, int32_t d, int32_t bits, int32_t group,
@@ -304,6 +360,7 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   p.rows_all = static_cast<int64_t>(cache->B) * H_q * L_q;
   p.ws_o = nullptr;
   p.ws_lse = nullptr;
+  p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cache->key_block) {
     // bf16 inputs split the cached keys when the caller gave the workspace for it.
@@ -423,6 +480,15 @@ QKV_API qkv_status attention_fidelity(const void* Q, int32_t dtype, int32_t H_q,
   return QKV_OK;
 }
 
+QKV_API qkv_status qkv_set_wait_limit(int64_t cycles, int64_t* previous) {
+  t_last_error.clear();
+  if (cycles < 0) return fail(QKV_ERR_INVALID_ARG, "wait limit must be >= 0 (0 restores the default)");
+  const long long v = cycles == 0 ? kDefaultWaitLimitCycles : static_cast<long long>(cycles);
+  const long long old = g_wait_limit.exchange(v, std::memory_order_relaxed);
+  if (previous) *previous = old;
+  return QKV_OK;
+}
+
 QKV_API qkv_status qkv_device_status(int32_t reset, int32_t* code) {
   t_last_error.clear();
   if (!code) return fail(QKV_ERR_INVALID_ARG, "NULL output");
@@ -452,28 +518,16 @@ QKV_API qkv_status qkv_device_status(int32_t reset, int32_t* code) {
 //
 // In host code the array's name is only a host-side stand-in, not a device address: a kernel given
 // it would fault or, where the GPU can reach host memory, silently use the wrong memory. Its device
-// address is therefore looked up with cudaGetSymbolAddress, once per device with that device
-// current (on the entry point's first call on the device that needs the scratch), and passed to
-// the kernels.
+// address is therefore looked up with cudaGetSymbolAddress, with that device current, on the entry
+// point's first call on the device that needs the scratch (and again if the device's context has
+// been re-created since), and passed to the kernels.
 static constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
+static SymbolAddressCache g_scratch_addr;
+
 static float* noalloc_scratch(cudaError_t* err) {
-  static float* addr[64] = {nullptr};
-  int dev = 0;
-  *err = cudaGetDevice(&dev);
-  if (*err != cudaSuccess) return nullptr;
-  if (dev < 0 || dev >= 64) {
-    *err = cudaErrorInvalidDevice;
-    return nullptr;
-  }
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (*err != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<float*>(p);
-  }
-  return addr[dev];
+  return static_cast<float*>(symbol_address(g_scratch_addr, g_noalloc_scratch, err));
 }
 
 QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
@@ -501,14 +555,14 @@ QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int
   const int64_t rows = static_cast<int64_t>(H_q / cache->H_kv) * L_q;
   if ((rows + 127) / 128 > 2147483647LL || static_cast<int64_t>(cache->B) * cache->H_kv > 65535)
     return fail(QKV_ERR_UNSUPPORTED, "grid too large");
-  // The key split this shape takes, and whether its scratch fits the library's array.
-  const int n = dtype == QKV_BF16 && !cache->key_block ? attention_splits(cache, H_q, L_q) : 1;
-  const size_t need = split_workspace_bytes(cache, H_q, L_q, n);
-  if (need > kNoAllocScratchBytes)
-    return fail(QKV_ERR_UNSUPPORTED,
-                "this shape splits its cached keys %d ways and needs %zu bytes of scratch; the "
-                "library's static scratch holds %zu bytes (use corrected_attention with a workspace)",
-                n, need, kNoAllocScratchBytes);
+  // The key split this shape takes, cut down to as many splits as the library's array holds the
+  // partials of; fewer than two run unsplit (the same result, with fewer CTAs sharing the reads).
+  int n = dtype == QKV_BF16 && !cache->key_block ? attention_splits(cache, H_q, L_q) : 1;
+  if (n > 1) {
+    const size_t per_split = split_workspace_bytes(cache, H_q, L_q, 2) / 2;
+    const size_t fit = kNoAllocScratchBytes / per_split;
+    if (fit < static_cast<size_t>(n)) n = fit >= 2 ? static_cast<int>(fit) : 1;
+  }
   cudaError_t e;
   int* status = status_word(&e);
   if (!status) return cuda_fail(e, "device status word");
@@ -537,6 +591,7 @@ QKV_API qkv_status corrected_attention_noalloc(const void* Q, int32_t dtype, int
   p.rows_all = static_cast<int64_t>(cache->B) * H_q * L_q;
   p.ws_o = scratch;
   p.ws_lse = scratch ? scratch + static_cast<size_t>(n) * p.rows_all * cache->d : nullptr;
+  p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   e = cache->key_block ? launch_attention_channel(p, cache->d, cache->bits, cache->key_block, st)
       : dtype == QKV_F32 ? launch_attention_f32(p, cache->d, cache->bits, st)

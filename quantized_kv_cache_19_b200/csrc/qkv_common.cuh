@@ -9,7 +9,9 @@
 
 namespace qkv {
 
-// A bounded wait gives up after this many SM clock cycles (about a second at 1.9 GHz).
+// Default bound of a wait, in SM clock cycles (about a second at 1.9 GHz). Kernels take the bound
+// of their progress waits from their parameters (the host can lower it to test the timeout path);
+// the waits on the way out of a kernel (outstanding copies and MMAs) always use this one.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -44,7 +46,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed. Gives up (returns false) when the
-// CTA-wide abort flag is raised by another thread, or after kWaitLimitCycles, in which case it
+// CTA-wide abort flag is raised by another thread, or after `limit` cycles, in which case it
 // raises the abort flag and records QKV_ERR_TIMEOUT (-5) in the device status word `status`
 // (the library's word, 0 while no error has been seen).
 // try_wait with a suspend-time hint: the thread sleeps in hardware until the phase completes (it is
@@ -62,13 +64,13 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       atomicCAS(status, 0, -5);
       return false;
@@ -78,8 +80,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Warp-uniform form: every lane polls; the warp proceeds only if every lane saw the phase, so a
 // timeout never splits the warp before a warp-collective instruction.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status));
+                                          int* status, long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, status, limit));
+}
+// Named barrier over `nthreads` threads that also ORs a per-thread flag over them: every thread
+// gets true if any participant passed true. Lets a group of warps that share named barriers decide
+// together to leave a loop, so that all of them execute the same sequence of barriers.
+__device__ __forceinline__ bool named_sync_or(int id, int nthreads, bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(flag)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 // Bounded wait used on the way out of a kernel: ignores the abort flag, never records an error.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
@@ -88,6 +105,72 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
   return true;
+}
+
+// Wait on the way out of a kernel for a phase completed from elsewhere (e.g. by a tensor-core
+// commit of the peer CTA), sleeping in hardware between polls: ignores the abort flag, records no
+// error, gives up after kWaitLimitCycles.
+__device__ __forceinline__ bool mbar_wait_drain_sleep(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait_sleep(bar, parity, 20000u)) {
+    if (clock64() - t0 > kWaitLimitCycles) return false;
+  }
+  return true;
+}
+
+// ------------------------------------------------------------------ clusters (CTA pairs)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster; release/acquire orders shared-memory writes.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared::cluster address of the same shared-memory offset in CTA `cta` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(cta));
+  return r;
+}
+// Arrive on an mbarrier of any CTA of the cluster (a shared::cluster address), releasing this
+// thread's earlier writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void st_shared_cluster(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// try_wait with cluster-scope acquire: for phases completed by arrivals from the peer CTA, whose
+// shared-memory and tensor-memory writes must be visible to what this thread issues next.
+__device__ __forceinline__ bool mbar_try_wait_sleep_cluster(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P1, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+// mbar_wait for phases completed from the peer CTA of a pair (cluster-scope acquire). On timeout
+// it also raises the peer's abort flag (`peer_abort`, a shared::cluster address).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* status, long long limit, uint32_t peer_abort) {
+  if (mbar_try_wait_sleep_cluster(bar, parity, 0u)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_sleep_cluster(bar, parity, 1000u)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) {
+      *abort_flag = 1;
+      st_shared_cluster(peer_abort, 1u);
+      atomicCAS(status, 0, -5);
+      return false;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ bulk copies (TMA engine)
@@ -107,6 +190,52 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // ------------------------------------------------------------------ tcgen05 / tensor memory
+// CTA-pair forms (cta_group::2): allocation and release are issued by the same warp of both CTAs
+// of the pair; an MMA is issued by one thread of the even CTA and computes M = 256 rows, 128 in
+// each CTA's tensor memory, with the B operand split along N between the two CTAs' shared memory
+// (the first half in the even CTA) at the same offsets. Every tcgen05 instruction of a kernel uses
+// the same cta_group.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// Arrives once on the mbarrier at this offset in every CTA of `cta_mask` when the pair MMAs issued
+// so far by this thread are done.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(cta_mask)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+      "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
+      "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
                "r"(ncols)

@@ -9,6 +9,9 @@ namespace qkv {
 
 enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 
+// Default bound of a kernel's progress waits, in SM clock cycles (about a second at 1.9 GHz).
+constexpr long long kDefaultWaitLimitCycles = 2000000000LL;
+
 // Quantise-and-append: K and V [B][H_kv][L_new][d] into the cache at positions start..start+L_new-1.
 struct QuantAppendParams {
   const void* K;
@@ -54,6 +57,7 @@ struct AttnParams {
   int64_t rows_all;     // B * Hq * Lq
   float* ws_o;
   float* ws_lse;
+  long long wait_limit;   // bound of the kernel's progress waits, SM clock cycles
 };
 // bf16 inputs: tcgen05 kernel. fp32 inputs: CUDA-core fp32 kernel.
 cudaError_t launch_attention_bf16(const AttnParams& p, int d, int bits, cudaStream_t stream);

@@ -166,3 +166,23 @@ def test_key_block_rejections(lib):
     st = P(0x80000)
     assert lib.attention_fidelity(P(0x70000), api.QKV_BF16, 2, 0, ctypes.byref(c2), P(0xA0000), None, 0,
                                   1, 0, 0.0, st, None, None) == 0
+
+
+def test_symbol_address_cache_policy(tmp_path):
+    """The remembered device addresses of the library's own device variables (the status word and
+    the allocation-free entry point's scratch) are reused only in the CUDA context they were looked
+    up in, and the cache is safe across host threads: a host-only C++ test of the helper."""
+    import os
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("g++ not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = str(tmp_path / "symbol_cache_test")
+    subprocess.run([gxx, "-std=c++17", "-O1", "-pthread",
+                    "-I" + os.path.join(root, "quantized_kv_cache_19_b200", "csrc"),
+                    os.path.join(root, "tests", "native", "symbol_cache_test.cpp"), "-o", exe],
+                   check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout + r.stderr
