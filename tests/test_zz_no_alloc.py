@@ -53,9 +53,10 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(Lq):
 
 
 def test_noalloc_splits_fewer_ways_when_the_workspace_split_does_not_fit():
-    # 4 x 8 KV heads, 128 query rows each: the workspace split (4 ways) needs 8.45 MB of partials,
-    # more than the 8 MiB array; the allocation-free call then splits 3 ways, with the same results
-    w = WORKLOADS["prefill_gqa"].with_(Lq=32, Lcur=32, Lc=2048 + 40, seed=901)
+    # 2 KV heads, 256 query rows each (one CTA pair per KV head): the workspace split (32 ways)
+    # needs 8.45 MB of partials, more than the 8 MiB array; the allocation-free call then splits
+    # 31 ways, with the same results
+    w = WORKLOADS["prefill_gqa"].with_(B=1, Hq=8, Hkv=2, Lq=64, Lcur=64, Lc=4096 + 40, seed=901)
     x, cache = _problem(w)
     assert api.attention_workspace_bytes(cache, w.Hq, w.Lq, w.Lcur) > STATIC_SCRATCH_BYTES
     O_ref, L_ref = _run(w, api.corrected_attention, x, cache)
