@@ -248,8 +248,10 @@ QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const voi
 }
 
 // Splits of the cached keys for the bf16 kernel: used only when the (row tile, batch * KV head)
-// grid would leave more than half of the SMs idle (few query rows per KV head, e.g. decoding);
-// each split then keeps at least one key tile. 1 = no split.
+// grid would leave more than half of the SMs idle (few query rows per KV head, e.g. decoding). The
+// kernel runs one CTA per SM, so the split count is the one whose grid fills whole waves of the
+// SMs best (the smallest such), at most 32 (the merge's limit) and at most one split per key tile.
+// 1 = no split.
 static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
   if (L_q <= 0 || c->length <= 0) return 1;
   int dev = 0, sms = 148;
@@ -263,10 +265,17 @@ static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
   const int tile = attention_tile_keys(c->d / c->group);
   const int64_t tiles = (c->length + tile - 1) / tile;
   if (ctas * 2 > sms || tiles < 2) return 1;
-  int64_t n = sms / ctas;
-  if (n > tiles) n = tiles;
-  if (n > 32) n = 32;
-  return n < 1 ? 1 : static_cast<int>(n);
+  int best = 1;
+  double best_fill = -1.0;
+  for (int n = 1; n <= 32 && n <= tiles; ++n) {
+    const int64_t grid = ctas * n;
+    const double fill = static_cast<double>(grid) / static_cast<double>(((grid + sms - 1) / sms) * sms);
+    if (fill > best_fill + 1e-9) {
+      best_fill = fill;
+      best = n;
+    }
+  }
+  return best;
 }
 
 // Splits of the cached keys for the per-channel-key kernel (bf16 inputs): as for the tensor-core
