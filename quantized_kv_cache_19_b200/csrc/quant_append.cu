@@ -85,7 +85,8 @@ __device__ __forceinline__ uint32_t pack_codes8(const float (&x)[8], float zp, f
 #pragma unroll
   for (int k = 0; k < 8; k += 2) {
     // The product stays a separately rounded multiply (__fmul_rn is never merged into an FMA): a
-    // fused multiply-add with the rounding constant would round exact ties the wrong way.
+    // fused multiply-add with the rounding constant would round exact ties the wrong way. (The
+    // pair form __fmul2_rn changed the codes of exact ties, so the two products stay scalar.)
     const float2 dx = __fadd2_rn(make_float2(x[k], x[k + 1]), nzp);
     float2 v = make_float2(__fmul_rn(dx.x, inv), __fmul_rn(dx.y, inv));
     if (kClamp) {
@@ -126,12 +127,16 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock + pr;
 
   for (int64_t bh = blockIdx.y; bh < p.BH; bh += gridDim.y) {
+    // This thread's first row and channels of the block; row u of the passes is u * kRowsPerPass
+    // rows further on (constant strides).
+    const InT* src = src_base + (bh * p.L_new + t0) * D + lr * 8;
+    const int64_t dst_row0 = bh * p.capacity + p.start + t0;
     float x[kPasses][8];
 #pragma unroll
     for (int u = 0; u < kPasses; ++u) {
       const int64_t t = t0 + u * kRowsPerPass;
       if (t < p.L_new) {
-        load8(src_base + (bh * p.L_new + t) * D + lr * 8, x[u]);
+        load8(src + u * kRowsPerPass * D, x[u]);
       } else {
 #pragma unroll
         for (int k = 0; k < 8; ++k) x[u][k] = 0.f;
@@ -167,7 +172,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
     {
       const int64_t t = t0 + uo * kRowsPerPass;
       if (jg < kPasses && t < p.L_new) {
-        const int64_t dst_row = bh * p.capacity + p.start + t;
+        const int64_t dst_row = dst_row0 + uo * kRowsPerPass;
         MetaOps<MetaT>::put_pair(meta_base + (dst_row * kNG + lr / kTpg) * 2, step_m, zp_m);
       }
     }
@@ -179,8 +184,7 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const QuantAppendP
       const int64_t t = t0 + u * kRowsPerPass;
       if (t >= p.L_new) continue;
       const uint32_t packed = pack_codes8<BITS, !std::is_same<MetaT, float>::value>(x[u], zp, inv);
-      const int64_t dst_row = bh * p.capacity + p.start + t;
-      uint8_t* codes = codes_base + dst_row * (D * BITS / 8) + lr * BITS;
+      uint8_t* codes = codes_base + (dst_row0 + u * kRowsPerPass) * (D * BITS / 8) + lr * BITS;
       if (BITS == 2) {
         *reinterpret_cast<uint16_t*>(codes) = static_cast<uint16_t>(packed);
       } else {
