@@ -56,7 +56,7 @@ def load_peaks():
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 CSRC = os.path.join(ROOT, "quantized_kv_cache_19_b200", "csrc")
 KERNEL_SOURCES = {
-    "corrected_attention_kernel": ["attention.cu", "qkv_common.cuh", "qkv_jensen.cuh", "qkv_internal.h"],
+    "corrected_attention_kernel": ["attention.cu", "qkv_common.cuh", "qkv_jensen.cuh", "qkv_internal.h", "tile_ops.cuh"],
     "quantize_append_kernel": ["quant_append.cu", "qkv_common.cuh", "qkv_internal.h"],
     "attention_fidelity_kernel": ["fidelity.cu", "fidelity.h", "qkv_common.cuh", "qkv_jensen.cuh"],
 }
@@ -518,6 +518,9 @@ def e2e_leg(w, x, cache, dev, flush, n_steps: int):
 
 def run_ours(args, world, rank, local):
     w_full = w = WORKLOADS[args.workload]
+    if args.cache_tokens is not None:
+        # the same shape with a shorter cache: small enough for a profiler capture of one launch
+        w_full = w = w.with_(Lc=args.cache_tokens)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     peaks, peak_kind = load_peaks()
@@ -705,6 +708,8 @@ def main(argv=None):
     ap.add_argument("--no-fidelity", action="store_true", help="skip the attention-fidelity diagnostics")
     ap.add_argument("--no-key-channel", action="store_true", help="skip the per-channel key layout leg")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' figures")
+    ap.add_argument("--cache-tokens", type=int, default=None,
+                    help="override the workload's cache length (for profiler captures of a smaller case)")
     ap.add_argument("--split-heads", action="store_true",
                     help="with several ranks: split one problem by (batch, KV head) instead of replicas")
     ap.add_argument("--record-traffic", metavar="NCU_REP", default=None,
