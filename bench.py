@@ -407,15 +407,18 @@ def fidelity_leg(dev, flush, steps: int = 10):
 
 def key_channel_leg(dev, flush, T: int = 32, steps: int = 10):
     """Per-channel keys along tokens (blocks of T positions, KIVI's group size of 32) on the bf16
-    INT2 workload: the whole-cache quantise-append (keys per channel, values per token; HBM-bound) and
-    corrected attention (correct=1) on the fp32 CUDA-core kernel that serves this layout, against
-    the fp32 FMA peak."""
+    INT2 workload: the whole-cache quantise-append (keys per channel, values per token; HBM-bound),
+    corrected attention with correct=1 on the tensor-core kernel for this layout (against the bf16
+    peak), and with correct=2 on the fp32 CUDA-core kernel that serves the fourth-order term
+    (against the fp32 FMA peak)."""
     w = WORKLOADS["bf16_int2"]
     x = make_inputs(w, device=dev)
     props = torch.cuda.get_device_properties(dev)
-    sm_mhz = float(load_peaks()[0].get("sm_max_mhz", 1965.0))
+    peaks = load_peaks()[0]
+    sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
     fp32_peak = props.multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
-    hbm = float(load_peaks()[0]["hbm_gbs"])
+    hbm = float(peaks["hbm_gbs"])
+    bf16_peak = float(peaks["bf16_tflops"])
     cache = api.KVCache(w.B, w.Hkv, w.d, w.bits, w.group, api.round_capacity(w.Lc), w.meta, device=dev,
                         key_block=T)
     stream = torch.cuda.current_stream(dev)
@@ -429,24 +432,28 @@ def key_channel_leg(dev, flush, T: int = 32, steps: int = 10):
     q_bytes = 2 * w.B * w.Hkv * w.Lc * w.d * in_bytes + cache.packed_bytes(w.Lc)
     O = torch.empty_like(x["Q"])
     LSE = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
-    a_ms = timed_ms(lambda: api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1,
-                                                    causal=w.causal, out=O, lse=LSE), stream, flush, steps)
-    if api.device_status() != 0:
-        raise RuntimeError("device status after the per-channel key leg")
     flops = api.attention_flops(w.B, w.Hq, w.Lq, w.Lc, w.Lcur, w.d, w.causal)
-    tf = flops / (a_ms * 1e-3) / 1e12
-    gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    out = {"workload": describe(w), "key_block": T,
+           "quantize_append_full_cache": {"bound": "hbm", "ms": round(q_ms, 4), "bytes": q_bytes,
+                                          "achieved_gbs": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+                                          "peak_gbs": hbm,
+                                          "frac": round(q_bytes / (q_ms * 1e-3) / 1e9 / hbm, 4)}}
+    for correct, key, kernel, bound, peak, kind in (
+            (1, "attention", "chan_attention_kernel (tensor cores)", "tensor", bf16_peak,
+             "bf16 dense, of measured"),
+            (2, "attention_correct2", "attention_f32_kernel (per-channel keys, CUDA cores)", "alu",
+             fp32_peak, "fp32 FMA: SMs x 128 lanes x 2 x max SM clock")):
+        a_ms = timed_ms(lambda: api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=correct,
+                                                        causal=w.causal, out=O, lse=LSE), stream, flush, steps)
+        if api.device_status() != 0:
+            raise RuntimeError("device status after the per-channel key leg")
+        tf = flops / (a_ms * 1e-3) / 1e12
+        out[key] = {"kernel": kernel, "correct": correct, "bound": bound, "ms_per_launch": round(a_ms, 4),
+                    "flops_per_launch": flops, "achieved": round(tf, 2), "peak": round(peak, 1),
+                    "unit": "TFLOP/s", "peak_kind": kind, "frac": round(tf / peak, 4)}
     del cache, x
     torch.cuda.empty_cache()
-    return {"workload": describe(w), "key_block": T,
-            "quantize_append_full_cache": {"bound": "hbm", "ms": round(q_ms, 4), "bytes": q_bytes,
-                                           "achieved_gbs": round(gbs, 1), "peak_gbs": hbm,
-                                           "frac": round(gbs / hbm, 4)},
-            "attention": {"kernel": "attention_f32_kernel (per-channel keys)", "bound": "alu",
-                          "ms_per_launch": round(a_ms, 4), "flops_per_launch": flops,
-                          "achieved": round(tf, 2), "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
-                          "peak_kind": "fp32 FMA: SMs x 128 lanes x 2 x max SM clock",
-                          "frac": round(tf / fp32_peak, 4)}}
+    return out
 
 
 def e2e_leg(w, x, cache, dev, flush, n_steps: int):

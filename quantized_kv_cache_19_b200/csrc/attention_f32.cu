@@ -397,6 +397,7 @@ int channel_rows_per_cta() { return kRows; }
 int channel_tile_keys() { return kKT; }
 
 cudaError_t launch_attention_channel(const AttnParams& p, int d, int bits, int T, cudaStream_t stream) {
+  if (chan_tc_serves(d, p.in_f32, p.correct)) return launch_attention_channel_tc(p, bits, T, stream);
   if (p.in_f32) {
     return d == 128 ? launch_f32<128, true, true>(p, bits, T, stream)
                     : launch_f32<64, true, true>(p, bits, T, stream);

@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <string>
@@ -247,12 +248,12 @@ QKV_API qkv_status kv_quantize_append(qkv_cache* cache, const void* K, const voi
   return QKV_OK;
 }
 
-// Splits of the cached keys for the bf16 kernel: used only when the (row tile, batch * KV head)
-// grid would leave more than half of the SMs idle (few query rows per KV head, e.g. decoding). The
-// kernel runs one CTA per SM, so the split count is the one whose grid fills whole waves of the
-// SMs best (the smallest such), at most 32 (the merge's limit) and at most one split per key tile.
-// 1 = no split.
-static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
+// Splits of the cached keys for the tensor-core kernels: used only when the (row tile, batch * KV
+// head) grid of 128-row CTAs would leave more than half of the SMs idle (few query rows per KV
+// head, e.g. decoding). The kernels run one CTA per SM, so the split count is the one whose grid
+// fills whole waves of the SMs best (the smallest such), at most 32 (the merge's limit) and at most
+// one split per key tile of `tile` keys. 1 = no split.
+static int wave_splits(const qkv_cache* c, int32_t H_q, int64_t L_q, int tile) {
   if (L_q <= 0 || c->length <= 0) return 1;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -262,7 +263,6 @@ static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
   }
   const int64_t rows = static_cast<int64_t>(H_q / c->H_kv) * L_q;
   const int64_t ctas = (rows + 127) / 128 * c->B * c->H_kv;
-  const int tile = attention_tile_keys(c->d / c->group);
   const int64_t tiles = (c->length + tile - 1) / tile;
   if (ctas * 2 > sms || tiles < 2) return 1;
   int best = 1;
@@ -278,11 +278,17 @@ static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
   return best;
 }
 
-// Splits of the cached keys for the per-channel-key kernel (bf16 inputs): as for the tensor-core
-// kernel, only when the (row tile, batch * KV head) grid would leave more than half of the SMs idle
-// (few query rows per KV head). Splitting fuller grids was measured slower: this CUDA-core kernel
-// gains nothing from a second CTA on an SM. 1 = no split.
-static int channel_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
+static int attention_splits(const qkv_cache* c, int32_t H_q, int64_t L_q) {
+  return wave_splits(c, H_q, L_q, attention_tile_keys(c->d / c->group));
+}
+
+// Splits of the cached keys for the per-channel-key kernels (bf16 inputs). The tensor-core kernel
+// (`tc`) splits like the per-token one. The CUDA-core kernel splits only when the (row tile,
+// batch * KV head) grid would leave more than half of the SMs idle, into as many splits as fit one
+// wave: splitting fuller grids was measured slower, as that kernel gains nothing from a second CTA
+// on an SM. 1 = no split.
+static int channel_splits(const qkv_cache* c, int32_t H_q, int64_t L_q, bool tc) {
+  if (tc) return wave_splits(c, H_q, L_q, kChanTcTileKeys);
   if (L_q <= 0 || c->length <= 0) return 1;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -315,8 +321,13 @@ QKV_API qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, i
   if (!bytes) return fail(QKV_ERR_INVALID_ARG, "NULL output");
   if (H_q < 1 || H_q % cache->H_kv || L_q < 0 || L_cur < 0)
     return fail(QKV_ERR_INVALID_ARG, "bad H_q / L_q / L_cur");
-  // The per-channel-key kernel splits only bf16 inputs; this size covers them (fp32 inputs ignore it).
-  const int n = cache->key_block ? channel_splits(cache, H_q, L_q) : attention_splits(cache, H_q, L_q);
+  // The per-channel-key kernels split only bf16 inputs; this size covers both of them (the
+  // tensor-core one serves correct <= 1, the CUDA-core one the rest; fp32 inputs ignore it).
+  int n = attention_splits(cache, H_q, L_q);
+  if (cache->key_block) {
+    n = channel_splits(cache, H_q, L_q, false);
+    if (chan_tc_serves(cache->d, 0, 0)) n = std::max(n, channel_splits(cache, H_q, L_q, true));
+  }
   *bytes = split_workspace_bytes(cache, H_q, L_q, n);
   return QKV_OK;
 }
@@ -373,7 +384,8 @@ QKV_API qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cache->key_block) {
     // bf16 inputs split the cached keys when the caller gave the workspace for it.
-    const int n = dtype == QKV_BF16 ? channel_splits(cache, H_q, L_q) : 1;
+    const bool tc = chan_tc_serves(cache->d, dtype == QKV_F32, correct);
+    const int n = dtype == QKV_BF16 ? channel_splits(cache, H_q, L_q, tc) : 1;
     const size_t need = split_workspace_bytes(cache, H_q, L_q, n);
     if (n > 1 && workspace && workspace_bytes >= need && aligned16(workspace)) {
       p.n_split = n;

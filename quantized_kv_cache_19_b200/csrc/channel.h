@@ -33,6 +33,13 @@ cudaError_t launch_attention_channel(const AttnParams& p, int d, int bits, int T
 int channel_rows_per_cta();
 int channel_tile_keys();
 
+// The tensor-core kernel for per-channel key blocks (attention_chan.cu) serves d = 128, bf16
+// inputs and correct <= 1; launch_attention_channel routes those calls to it. It takes 128 query
+// rows per CTA and 128-key tiles; with p.n_split > 1 it splits the 128-key tiles of the cache.
+bool chan_tc_serves(int d, int in_f32, int correct);
+constexpr int kChanTcTileKeys = 128;
+cudaError_t launch_attention_channel_tc(const AttnParams& p, int bits, int T, cudaStream_t stream);
+
 // Correction term alone over per-channel key blocks: bias[B][Hq][Lq][Lc].
 cudaError_t launch_jensen_bias_channel(const BiasParams& p, int T, cudaStream_t stream);
 
