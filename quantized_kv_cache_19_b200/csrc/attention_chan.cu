@@ -7,7 +7,7 @@
 // zero-point, so the per-token code-domain identity of the 128-row kernel does not apply (its scale
 // a_jg multiplies a whole group of one key; here every channel has its own). The keys are therefore
 // dequantised in fp32, x_hat = zp_c + step_c * code, and split into two bf16 tiles, high and low
-// (x_hat = hi + lo to ~2^-16 relative): S = Q K_hi^T + Q K_lo^T in one fp32 accumulator, two
+// (x_hat = hi + lo to ~2^-14 relative): S = Q K_hi^T + Q K_lo^T in one fp32 accumulator, two
 // chains of eight 128 x 128 x 16 MMAs with both operands in shared memory. The correction of the
 // Jensen-bias pages (agents-report.net, section 方法) is the same for all keys of a block:
 // b = (scale^2 / 24) sum_c q_c^2 step_c^2, taken for the 128 / T blocks of a tile by MMAs of
@@ -44,8 +44,9 @@ constexpr int kBM = 128;                      // query rows per CTA (MMA M)
 constexpr int kN = 128;                       // keys per tile
 constexpr int kThreads = 640;
 constexpr int kKThreads = 224;                // K producers: warps 1-3 and warpgroup 4
-// Registers per thread after setmaxnreg: 2 * 128 * 144 + 3 * 128 * 64 = 61440 = 640 * 96.
-constexpr int kRegProducer = 64, kRegSoftmax = 144;
+// Registers per thread after setmaxnreg: 2 * 128 * 128 + 3 * 128 * 72 = 60416 <= 640 * 96, the
+// block's allocation at launch (the producers' dequantisation spills at 64).
+constexpr int kRegProducer = 72, kRegSoftmax = 128;
 constexpr int kStagesMax = 3;                // packed-tile ring (INT2: 3 stages, INT4: 2)
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kTmemCols = 512;
@@ -55,8 +56,8 @@ constexpr int kCRows = 16;
 
 enum {
   B_PK_FULL = 0, B_PK_EMPTY = B_PK_FULL + kStagesMax,
-  B_KH_FULL = B_PK_EMPTY + kStagesMax, B_KH_EMPTY = B_KH_FULL + 1,
-  B_VH_FULL = B_KH_EMPTY + 1, B_VH_EMPTY = B_VH_FULL + 2,
+  B_KH_FULL = B_PK_EMPTY + kStagesMax, B_KH_EMPTY = B_KH_FULL + 2,   // per 64-channel half
+  B_VH_FULL = B_KH_EMPTY + 2, B_VH_EMPTY = B_VH_FULL + 2,
   B_S_FULL = B_VH_EMPTY + 2, B_S_FREE = B_S_FULL + 1,
   B_P_FULL = B_S_FREE + 1, B_PV_DONE = B_P_FULL + 1,
   B_Q_FULL = B_PV_DONE + 1, B_DRAIN = B_Q_FULL + 1,
@@ -97,16 +98,6 @@ __host__ __device__ inline CLayout make_clayout(int meta_bytes, int T) {
   return L;
 }
 
-// Eight channels of a key's packed codes (16 bits at INT2, 32 at INT4; channel k at bits k * BITS)
-// as exact floats.
-template <int BITS>
-__device__ __forceinline__ void codes8(uint32_t w, float (&c)[8]) {
-  constexpr uint32_t kMask = (1u << BITS) - 1u;
-#pragma unroll
-  for (int k = 0; k < 8; ++k)
-    c[k] = __uint_as_float(0x4B000000u | ((w >> (k * BITS)) & kMask)) - 8388608.0f;
-}
-
 // (step, zero-point) of 8 consecutive channels of a block's meta [D][2].
 template <bool F16>
 __device__ __forceinline__ void meta8(const uint8_t* meta, int c0, float (&st)[8], float (&zp)[8]) {
@@ -130,10 +121,58 @@ __device__ __forceinline__ void meta8(const uint8_t* meta, int c0, float (&st)[8
   }
 }
 
+// Dequantisation of one 8-channel chunk of a key block, x = zp + step * code, in the form
+// x = s' * (1 + code * 2^-k) + c' with s' = 2^k step and c' = zp - s': after one shift of the packed
+// codes word, the codes of a channel pair sit in the mantissa of 1.0 at bits 19-20 and 21-22 (INT2:
+// k = 4 and 2) or 15-18 and 19-22 (INT4: k = 8 and 4), so a pair is two masks and one paired FMA.
+struct ChunkScale {
+  float2 s[4], c[4];
+};
+template <int BITS, bool F16>
+__device__ __forceinline__ void chunk_scale(const uint8_t* meta, int c0, ChunkScale& cs);
+template <int BITS>
+__device__ __forceinline__ void dequant8_split(uint32_t w, const ChunkScale& cs, uint32_t (&hw)[4],
+                                               uint32_t (&lw)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t a, b;
+    if (BITS == 2) {
+      const uint32_t sh = w << (19 - 4 * q);
+      a = (sh & (3u << 19)) | 0x3F800000u;
+      b = (sh & (3u << 21)) | 0x3F800000u;
+    } else {
+      const int k = 15 - 8 * q;
+      const uint32_t sh = k >= 0 ? (w << k) : (w >> (-k));
+      a = (sh & (0xFu << 15)) | 0x3F800000u;
+      b = (sh & (0xFu << 19)) | 0x3F800000u;
+    }
+    const float2 x = __ffma2_rn(cs.s[q], make_float2(__uint_as_float(a), __uint_as_float(b)), cs.c[q]);
+    // hi = x truncated to bf16 (the upper halves of the two words), lo = the exact remainder x - hi
+    // truncated again: x = hi + lo to 2^-14 relative, with byte permutes and masks on the integer
+    // pipes instead of float-to-bf16 conversions.
+    const uint32_t ux = __float_as_uint(x.x), uy = __float_as_uint(x.y);
+    const float2 r = __fadd2_rn(x, make_float2(-__uint_as_float(ux & 0xFFFF0000u), -__uint_as_float(uy & 0xFFFF0000u)));
+    hw[q] = __byte_perm(ux, uy, 0x7632);
+    lw[q] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+  }
+}
+
 // One 16-byte chunk (8 channels) of row `row` into a [D/64][rows][64] bf16 tile, 128-byte swizzle.
 template <int ROWS>
 __device__ __forceinline__ void store_chunk(uint8_t* tile, int row, int chunk, uint4 v) {
   *reinterpret_cast<uint4*>(tile + (chunk >> 3) * (ROWS * 128) + sw128_offset(row, chunk & 7)) = v;
+}
+
+template <int BITS, bool F16>
+__device__ __forceinline__ void chunk_scale(const uint8_t* meta, int c0, ChunkScale& cs) {
+  float st[8], zp[8];
+  meta8<F16>(meta, c0, st, zp);
+  constexpr float kA = BITS == 2 ? 16.f : 256.f, kB = BITS == 2 ? 4.f : 16.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    cs.s[q] = make_float2(st[2 * q] * kA, st[2 * q + 1] * kB);
+    cs.c[q] = make_float2(zp[2 * q] - cs.s[q].x, zp[2 * q + 1] - cs.s[q].y);
+  }
 }
 
 template <int BITS, int NGV>
@@ -186,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
     *abort_flag = 0;
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_KH_FULL) cnt = kKThreads / 32;
+      if (i == B_KH_FULL || i == B_KH_FULL + 1) cnt = kKThreads / 32;
       if (i == B_VH_FULL || i == B_VH_FULL + 1) cnt = 4;
       if (i == B_S_FREE || i == B_P_FULL || i == B_Q_FULL) cnt = 8;   // both softmax warpgroups
       if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = kKThreads / 32 + 4;
@@ -236,17 +275,25 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
       bool ok = T_all > 0 && wait1(B_Q_FULL, 0);
       if (ok) tc_fence_after();
       for (int j = 0; j < T_all && ok; ++j) {
-        if (!wait1(B_KH_FULL, j & 1)) { ok = false; break; }
-        if (j >= 1 && !wait1(B_S_FREE, (j - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
         const bool cached = j < Tc;
+        // Each 64-channel half of the K tiles as soon as it is written: the producers write the
+        // second half of tile j while the first half's MMAs run.
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!wait1(B_KH_FULL + h, j & 1)) { ok = false; break; }
+          if (h == 0 && j >= 1 && !wait1(B_S_FREE, (j - 1) & 1)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kColS, qdesc + kofs(kk * 16), hdesc + kofs(kk * 16), idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+            mma_ss(tmem + kColS, qdesc + kofs(kk * 16), hdesc + kofs(kk * 16), idesc_s, kk > 0 ? 1u : 0u);
+          if (cached) {
+#pragma unroll
+            for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
+              mma_ss(tmem + kColS, qdesc + kofs(kk * 16), ldesc + kofs(kk * 16), idesc_s, 1u);
+          }
+          if (h == 0) tc_commit(bar(B_KH_EMPTY));
+        }
+        if (!ok) break;
         if (cached) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            mma_ss(tmem + kColS, qdesc + kofs(kk * 16), ldesc + kofs(kk * 16), idesc_s, 1u);
           if (p.correct) {
             // (q2_hi + q2_lo) x (rows blk: d2_hi, rows 4 + blk: d2_lo)
 #pragma unroll
@@ -257,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
               mma_ts(tmem + kColC, tmem + kColQ2L + kk * 8u, cdesc + cofs(kk * 16), idesc_c, 1u);
           }
         }
-        tc_commit(bar(B_KH_EMPTY));
+        tc_commit(bar(B_KH_EMPTY + 1));
         tc_commit(bar(B_S_FULL));
         if (j >= 1) ok = issue_pv(j - 1);
       }
@@ -270,92 +317,121 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
     // ---------------------------------------------------------------- K hi / lo tiles
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = wg == 0 ? threadIdx.x - 32 : threadIdx.x - 512 + 96;   // 0 .. kKThreads - 1
-    constexpr int kItems = kN * (D / 8);        // (key, 8-channel chunk) items of a tile
-    constexpr int kIters = (kItems + kKThreads - 1) / kKThreads;
+    // Half h of a tile is channels [64 h, 64 h + 64) of its hi and lo tiles. Thread t of warp
+    // w = t / 32 takes chunk cl of the half (8 channels) for the four keys of key lane
+    // 4 w + ks, [4 (4 w + ks), +4), which lie in one key block (T is a multiple of 4), in the order
+    // (i + ks) mod 4; threads of warps 0-3 also take one of the keys 112-127. A quarter-warp holds
+    // chunks {2 q, 2 q + 1} of four key lanes, so that its four rows and two chunks cover the eight
+    // 16-byte bank groups in every store of the swizzled tiles and in every load of the scales, and
+    // at INT2 its code loads fall in distinct banks. The four keys share one set of scales and no
+    // branch, so that their dequantisations interleave.
+    constexpr int kKeysA = 4;                   // 28 key lanes x 4 = 112 keys, then 16 x 1
+    static_assert((kKThreads / 8) * kKeysA + 128 / 8 == kN, "key lanes must cover a tile");
+    const int w7 = t >> 5, ks = (t & 7) >> 1;
+    const int cl = 2 * ((t & 31) >> 3) + (t & 1);
+    const int key0 = 4 * (4 * w7 + ks);
+    const int keyB = (kKThreads / 8) * kKeysA + 2 * ks + 8 * (w7 & 1) + (w7 >> 1);
+    const bool has_b = w7 < 4;
+    auto key_a = [&](int i) { return key0 + ((i + ks) & 3); };
+    const int tshift = __ffs(T) - 1;            // T is a power of two
     const int64_t row_codes = D * BITS / 8;
     uint8_t* khi = smem + L.khi;
     uint8_t* klo = smem + L.klo;
-    for (int j = 0; j < T_all; ++j) {
-      if (!waitw(B_KH_EMPTY, (j & 1) ^ 1)) break;
-      if (j < Tc) {
-        const int s = j % kStages;
+    bool kok = true;
+    for (int j = 0; j < T_all && kok; ++j) {
+      const bool cached = j < Tc;
+      const int s = j % kStages;
+      int valid;
+      if (cached) {
         const int64_t rem = p.Lc - static_cast<int64_t>(c0 + j) * kN;
-        const int valid = static_cast<int>(rem < kN ? rem : kN);
-        if (!waitw(B_PK_FULL + s, (j / kStages) & 1)) break;
-        const uint8_t* kcodes = smem + L.pk + s * L.stage;
-        const uint8_t* kmeta = kcodes + 2 * C::kCodes;          // [blocks][D][2]
-        const int mb = p.meta_f16 ? 2 : 4;
-#pragma unroll 1
-        for (int i = 0; i < kIters; ++i) {
-          // Item: 8 consecutive keys of one 8-channel chunk share the chunk's steps; consecutive
-          // threads take consecutive keys (conflict-free stores into the swizzled tiles).
-          const int it = t + kKThreads * i;
-          if (it >= kItems) break;
-          const int key = (it & 7) + ((it >> 3) / (D / 8)) * 8, chunk = (it >> 3) % (D / 8);
-          uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
-          if (key < valid) {
-            float st[8], zp[8], c[8];
-            const uint8_t* m = kmeta + (key / T) * D * 2 * mb;
-            if (p.meta_f16) meta8<true>(m, chunk * 8, st, zp);
-            else meta8<false>(m, chunk * 8, st, zp);
-            uint32_t w;
-            if (BITS == 2) w = *reinterpret_cast<const uint16_t*>(kcodes + key * row_codes + chunk * 2);
-            else w = *reinterpret_cast<const uint32_t*>(kcodes + key * row_codes + chunk * 4);
-            codes8<BITS>(w, c);
-#pragma unroll
-            for (int k = 0; k < 8; k += 2) {
-              const float2 x = __ffma2_rn(make_float2(st[k], st[k + 1]), make_float2(c[k], c[k + 1]),
-                                          make_float2(zp[k], zp[k + 1]));
-              const uint32_t hi = pack_bf16x2(x.x, x.y);
-              const float2 r = __fadd2_rn(x, make_float2(-bf16_lo(hi), -bf16_hi(hi)));
-              hw[k / 2] = hi;
-              lw[k / 2] = pack_bf16x2(r.x, r.y);
-            }
-          }
-          store_chunk<kN>(khi, key, chunk, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-          store_chunk<kN>(klo, key, chunk, make_uint4(lw[0], lw[1], lw[2], lw[3]));
-        }
-        // The tile's blocks' squared steps, scaled to the correction in log2 units.
-        if (p.correct && t < nblk * (D / 8)) {
-          const int blk = t / (D / 8), chunk = t % (D / 8);
-          float st[8], zp[8];
-          const uint8_t* m = kmeta + blk * D * 2 * mb;
-          if (p.meta_f16) meta8<true>(m, chunk * 8, st, zp);
-          else meta8<false>(m, chunk * 8, st, zp);
-          uint32_t ch[4], cl[4];
-#pragma unroll
-          for (int k = 0; k < 8; k += 2) {
-            const float2 d2 = __fmul2_rn(__fmul2_rn(make_float2(st[k], st[k + 1]), make_float2(st[k], st[k + 1])),
-                                         make_float2(p.wcoef_log2, p.wcoef_log2));
-            ch[k / 2] = pack_bf16x2(d2.x, d2.y);
-            const float2 r = __fadd2_rn(d2, make_float2(-bf16_lo(ch[k / 2]), -bf16_hi(ch[k / 2])));
-            cl[k / 2] = pack_bf16x2(r.x, r.y);
-          }
-          store_chunk<kCRows>(smem + L.ct, blk, chunk, make_uint4(ch[0], ch[1], ch[2], ch[3]));
-          store_chunk<kCRows>(smem + L.ct, 4 + blk, chunk, make_uint4(cl[0], cl[1], cl[2], cl[3]));
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(bar(B_KH_FULL));
-          mbar_arrive(bar(B_PK_EMPTY + s));
-        }
+        valid = static_cast<int>(rem < kN ? rem : kN);
       } else {
         const int64_t t0 = static_cast<int64_t>(j - Tc) * kN;
-        const int valid = static_cast<int>(cur_keys - t0 < kN ? cur_keys - t0 : kN);
+        valid = static_cast<int>(cur_keys - t0 < kN ? cur_keys - t0 : kN);
+      }
+      const uint8_t* kcodes = smem + L.pk + s * L.stage;
+      const uint8_t* kmeta = kcodes + 2 * C::kCodes;            // [blocks][D][2]
+      const int blk_bytes = D * 2 * (p.meta_f16 ? 2 : 4);
+      for (int h = 0; h < 2; ++h) {
+        if (!waitw(B_KH_EMPTY + h, (j & 1) ^ 1)) { kok = false; break; }
+        const int chunk = h * 8 + cl;
+        if (cached) {
+          if (h == 0 && !waitw(B_PK_FULL + s, (j / kStages) & 1)) { kok = false; break; }
+          auto load_code = [&](int key) -> uint32_t {
+            if (key >= valid) return 0u;
+            if (BITS == 2) return *reinterpret_cast<const uint16_t*>(kcodes + key * row_codes + chunk * 2);
+            return *reinterpret_cast<const uint32_t*>(kcodes + key * row_codes + chunk * 4);
+          };
+          auto scale_of = [&](int key, ChunkScale& cs) {
+            const uint8_t* m = kmeta + (key >> tshift) * blk_bytes;
+            if (p.meta_f16) chunk_scale<BITS, true>(m, chunk * 8, cs);
+            else chunk_scale<BITS, false>(m, chunk * 8, cs);
+          };
+          auto put = [&](int key, const uint32_t (&hw)[4], const uint32_t (&lw)[4]) {
+            const bool v = key < valid;          // keys past the cache end become zero
+            store_chunk<kN>(khi, key, chunk, v ? make_uint4(hw[0], hw[1], hw[2], hw[3]) : make_uint4(0u, 0u, 0u, 0u));
+            store_chunk<kN>(klo, key, chunk, v ? make_uint4(lw[0], lw[1], lw[2], lw[3]) : make_uint4(0u, 0u, 0u, 0u));
+          };
+          {
+            uint32_t w[kKeysA];
+#pragma unroll
+            for (int i = 0; i < kKeysA; ++i) w[i] = load_code(key_a(i));
+            ChunkScale cs;
+            scale_of(key0, cs);
+#pragma unroll
+            for (int i = 0; i < kKeysA; ++i) {
+              uint32_t hw[4], lw[4];
+              dequant8_split<BITS>(w[i], cs, hw, lw);
+              put(key_a(i), hw, lw);
+            }
+          }
+          if (has_b) {
+            const uint32_t wb = load_code(keyB);
+            ChunkScale cs;
+            scale_of(keyB, cs);
+            uint32_t hw[4], lw[4];
+            dequant8_split<BITS>(wb, cs, hw, lw);
+            put(keyB, hw, lw);
+          }
+          // The tile's blocks' squared steps, scaled to the correction in log2 units, as hi and lo
+          // parts (rows blk and 4 + blk), with the second half (read by the same MMAs).
+          // (Threads t >= 160, which have no fifth key.)
+          const int tc = t - (kKThreads - 64);
+          if (h == 1 && p.correct && tc >= 0 && tc < nblk * (D / 8)) {
+            const int blk = tc / (D / 8), ch = tc % (D / 8);
+            float st[8], zp[8];
+            if (p.meta_f16) meta8<true>(kmeta + blk * blk_bytes, ch * 8, st, zp);
+            else meta8<false>(kmeta + blk * blk_bytes, ch * 8, st, zp);
+            uint32_t dh[4], dl[4];
+#pragma unroll
+            for (int k = 0; k < 8; k += 2) {
+              const float2 d2 = __fmul2_rn(__fmul2_rn(make_float2(st[k], st[k + 1]), make_float2(st[k], st[k + 1])),
+                                           make_float2(p.wcoef_log2, p.wcoef_log2));
+              dh[k / 2] = pack_bf16x2(d2.x, d2.y);
+              const float2 r = __fadd2_rn(d2, make_float2(-bf16_lo(dh[k / 2]), -bf16_hi(dh[k / 2])));
+              dl[k / 2] = pack_bf16x2(r.x, r.y);
+            }
+            store_chunk<kCRows>(smem + L.ct, blk, ch, make_uint4(dh[0], dh[1], dh[2], dh[3]));
+            store_chunk<kCRows>(smem + L.ct, 4 + blk, ch, make_uint4(dl[0], dl[1], dl[2], dl[3]));
+          }
+        } else {
+          const int64_t t0 = static_cast<int64_t>(j - Tc) * kN;
+          const uint4* src = reinterpret_cast<const uint4*>(p.K_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
 #pragma unroll 1
-        for (int i = 0; i < kIters; ++i) {
-          const int it = t + kKThreads * i;
-          if (it >= kItems) break;
-          const int key = (it & 7) + ((it >> 3) / (D / 8)) * 8, chunk = (it >> 3) % (D / 8);
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (key < valid)
-            v = reinterpret_cast<const uint4*>(p.K_cur)[(static_cast<int64_t>(bh) * p.Lcur + t0 + key) * (D / 8) + chunk];
-          store_chunk<kN>(khi, key, chunk, v);
+          for (int i = 0; i <= kKeysA; ++i) {
+            if (i == kKeysA && !has_b) break;
+            const int key = i < kKeysA ? key_a(i) : keyB;
+            const uint4 v = key < valid ? src[key * (D / 8) + chunk] : make_uint4(0u, 0u, 0u, 0u);
+            store_chunk<kN>(khi, key, chunk, v);
+          }
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_KH_FULL));
+        if (lane == 0) mbar_arrive(bar(B_KH_FULL + h));
+      }
+      if (kok && cached) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PK_EMPTY + s));
       }
     }
   } else if (wg == 3) {
@@ -475,25 +551,29 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
       // This half's channels of Q (natural order) into shared memory, and of q^2 as two bf16 parts
       // (exact: q is bf16, so q^2 has at most 16 significant bits) into tensor memory.
       const uint8_t* qrow = static_cast<const uint8_t*>(p.Q) + out_row * D * 2;
-      uint32_t q2h[D / 4], q2l[D / 4];
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (valid_row) u = reinterpret_cast<const uint4*>(qrow)[half * (D / 16) + c];
-        store_chunk<kBM>(smem + L.qs, row, half * (D / 16) + c, u);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int g = 0; g < 2; ++g) {             // 32 channels (16 columns) at a time
+        uint32_t q2h[16], q2l[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 a = __fmul2_rn(make_float2(bf16_lo(w[e]), bf16_hi(w[e])), make_float2(bf16_lo(w[e]), bf16_hi(w[e])));
-          const uint32_t hi = pack_bf16x2(a.x, a.y);
-          const float2 r = __fadd2_rn(a, make_float2(-bf16_lo(hi), -bf16_hi(hi)));
-          q2h[4 * c + e] = hi;
-          q2l[4 * c + e] = pack_bf16x2(r.x, r.y);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int c = 4 * g + c4;
+          uint4 u = make_uint4(0u, 0u, 0u, 0u);
+          if (valid_row) u = reinterpret_cast<const uint4*>(qrow)[half * (D / 16) + c];
+          store_chunk<kBM>(smem + L.qs, row, half * (D / 16) + c, u);
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 a = __fmul2_rn(make_float2(bf16_lo(w[e]), bf16_hi(w[e])), make_float2(bf16_lo(w[e]), bf16_hi(w[e])));
+            const uint32_t hi = pack_bf16x2(a.x, a.y);
+            const float2 r = __fadd2_rn(a, make_float2(-bf16_lo(hi), -bf16_hi(hi)));
+            q2h[4 * c4 + e] = hi;
+            q2l[4 * c4 + e] = pack_bf16x2(r.x, r.y);
+          }
         }
+        tmem_st16(tmem + lane_off + kColQ2H + half * (D / 4) + 16 * g, q2h);
+        tmem_st16(tmem + lane_off + kColQ2L + half * (D / 4) + 16 * g, q2l);
       }
       fence_async_smem();
-      tmem_st<D / 4>(tmem + lane_off + kColQ2H + half * (D / 4), q2h);
-      tmem_st<D / 4>(tmem + lane_off + kColQ2L + half * (D / 4), q2l);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
