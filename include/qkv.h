@@ -145,10 +145,12 @@ qkv_status corrected_attention_workspace_bytes(const qkv_cache* cache, int32_t H
  *                 owned by the caller; NULL (or too small) runs the same attention without the
  *                 key split. Calls on one stream may reuse it; concurrent calls need their own.
  * L_cur = 0 and cache->length = 0 together are rejected (no keys at all).
- * A cache with per-channel keys (key_block > 0) is served by an fp32 CUDA-core kernel for bf16 and
- * fp32 inputs alike. With bf16 inputs it splits the cached keys over CTAs for decode-sized query
- * chunks (when the unsplit grid would leave more than half of the SMs idle) and then uses the
- * workspace the same way; fp32 inputs run unsplit and ignore the workspace.
+ * A cache with per-channel keys (key_block > 0) is served, for bf16 inputs with d = 128 and
+ * correct <= 1, by a tensor-core kernel that dequantises the keys into bf16 high and low parts, and
+ * otherwise (fp32 inputs, d = 64, correct = 2) by an fp32 CUDA-core kernel. With bf16 inputs both
+ * split the cached keys over CTAs for decode-sized query chunks (when the unsplit grid would leave
+ * more than half of the SMs idle) and then use the workspace the same way; fp32 inputs run unsplit
+ * and ignore the workspace. corrected_attention_workspace_bytes() covers either kernel.
  */
 qkv_status corrected_attention(const void* Q, int32_t dtype, int32_t H_q, int64_t L_q,
                                const qkv_cache* cache, const void* K_cur, const void* V_cur,
