@@ -27,7 +27,8 @@
 // warpgroups, registers rebalanced with setmaxnreg:
 //   WG0      warp 0: allocates tensor memory; one thread issues, in order, S_j = Q K_j^T and then
 //            P_{j-1} V_{j-1} with precomputed descriptors.
-//   WG0 warps 1-3 and WG4: K operand tiles (codes unpacked to exact bf16 integers, 128-byte
+//   WG0 warps 1-3 and the first 1-2 warps of WG4: K operand tiles (codes unpacked to exact bf16
+//            integers, 128-byte
 //            swizzle, two buffers) and the tile's per-key constants (scales a for the softmax, key
 //            extras for the S MMA); for current tiles, a copy of K_cur. Channels are stored in an
 //            operand order (k, k+8 interleaved inside each 16-channel block) that makes the unpack
@@ -37,7 +38,8 @@
 //            TMEM (releasing it at once), form the corrected scores, exchange the row max through
 //            shared memory, online softmax in base 2 with lazy rescaling of O (each half rescales
 //            half of O's columns), P (bf16) into TMEM; finally O / l and LSE.
-//   WG3      V operand tiles, dequantised to bf16; for current tiles, a copy of V_cur. One lane
+//   WG3 and the rest of WG4: V operand tiles, dequantised to bf16; for current tiles, a copy of
+//            V_cur (the split between K and V warps is in Cfg). One lane of WG3
 //            also issues the bulk (TMA-engine) copies of packed tiles (codes and step/zero-point
 //            of N keys, K and V) into a 2-3 stage ring.
 // Tensor memory (512 columns): O [0, d), Q [128, 128 + d/2), P [192, 256), S [256, 512) (one
@@ -57,7 +59,6 @@ namespace {
 
 constexpr int kBM = 128;                     // query rows per CTA (MMA M)
 constexpr int kThreads = 640;                 // five warpgroups
-constexpr int kKThreads = 224;                // K producers: warps 1-3 and warpgroup 4
 // Registers per thread after setmaxnreg: 2 * 128 * 144 + 3 * 128 * 64 = 61440 = 640 * 96, the
 // block's allocation at launch.
 constexpr int kRegProducer = 64, kRegSoftmax = 144;
@@ -97,6 +98,16 @@ struct Cfg {
   static constexpr int kSCols = NA * N;                  // TMEM columns of one S buffer
   static constexpr int kSB = 256 / kSCols;               // S buffers in the 256 S columns (1 or 2)
   static constexpr int kPB = 64 / (N / 2);               // P buffers in the 64 P columns (1 or 2)
+  // Producer warps: K on warps 1-3 and the first kKWarps - 3 warps of warpgroup 4, V on warpgroup 3
+  // and the rest of warpgroup 4 (11 in all). Warp w issues from sub-partition w % 4: with four K
+  // warps every sub-partition holds one K warp, two softmax warps and one or two V warps. Measured
+  // over 4-7 K warps (one launch each, 1965 MHz): 4 was fastest with two groups (chunked prefill
+  // 9.37 ms against 9.60 with 7), 5 with one group (the long-video cache 6.47 ms against 7.01);
+  // the V dequantisation costs more instructions than the K unpack and per-key constants.
+  static constexpr int kKWarps = NG == 1 ? 5 : 4;
+  static constexpr int kVWarps = 11 - kKWarps;
+  static constexpr int kKThreads = 32 * kKWarps;
+  static constexpr int kVThreads = 32 * kVWarps;
 };
 
 struct Layout {
@@ -163,13 +174,14 @@ __device__ __forceinline__ void copy_rows(const uint4* src, uint8_t* tile, int v
 template <int D, int BITS, int NG, bool kQuartic>
 __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const AttnParams p) {
   using C = Cfg<D, BITS, NG>;
+  constexpr int kKWarps = C::kKWarps, kVWarps = C::kVWarps;
+  constexpr int kKThreads = C::kKThreads, kVThreads = C::kVThreads;
   constexpr int N = C::N;
   constexpr int kStages = C::kStages;
   constexpr int NH = N / 2;                   // keys of a tile per softmax warpgroup
   constexpr int kItems = N * (D / 32);        // (key, 32-channel block) items of one tile
-  constexpr int kItersV = kItems / 128;       // per V-producer thread (128 threads)
+  constexpr int kItersV = (kItems + kVThreads - 1) / kVThreads;   // per V-producer thread
   constexpr int kItersK = (kItems + kKThreads - 1) / kKThreads;   // per K-producer thread
-  static_assert(kItems % 128 == 0 && kItersV % 2 == 0, "tile items must split evenly over a warpgroup");
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // 1024-byte alignment (128B-swizzle atoms) by offsetting the shared array itself, so that the
   // compiler keeps every access in the shared address space.
@@ -217,12 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     *abort_flag = 0;
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t cnt = 1;
-      if (i == B_KH_FULL || i == B_KH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1) cnt = 7;
-      if (i == B_VH_FULL || i == B_VH_FULL + 1) cnt = 4;
+      if (i == B_KH_FULL || i == B_KH_FULL + 1 || i == B_KC_FULL || i == B_KC_FULL + 1) cnt = kKWarps;
+      if (i == B_VH_FULL || i == B_VH_FULL + 1) cnt = kVWarps;
       if (i == B_KC_EMPTY || i == B_KC_EMPTY + 1 || i == B_S_FREE || i == B_S_FREE + 1 ||
           i == B_P_FULL || i == B_P_FULL + 1 || i == B_Q_FULL)
         cnt = 8;                                   // both softmax warpgroups
-      if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = 11;  // K and V producer warps
+      if (i >= B_PK_EMPTY && i < B_PK_EMPTY + kStages) cnt = kKWarps + kVWarps;  // K and V producer warps
       mbar_init(bar(i), cnt);
     }
     mbar_init_fence();
@@ -302,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       mbar_wait_drain(bar(B_DRAIN), 0);
     }
     __syncwarp();
-  } else if (wg == 0 || wg == 4) {
+  } else if (wg == 0 || (wg == 4 && warp < 16 + kKWarps - 3)) {
     // ---------------------------------------------------------------- K operand tiles (warps 1-3)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = wg == 0 ? threadIdx.x - 32 : threadIdx.x - 512 + 96;   // 0 .. kKThreads - 1
@@ -405,10 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         }
       }
     }
-  } else if (wg == 3) {
+  } else if (wg == 3 || wg == 4) {
     // ---------------------------------------------------------------- V operand tiles
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
-    const int t = threadIdx.x - 384;
+    const int t = wg == 3 ? threadIdx.x - 384 : threadIdx.x - 32 * (16 + kKWarps - 3) + 128;  // 0 .. kVThreads - 1
     // Lane 0 of the first V warp also issues the bulk copies of packed tiles, kStages - 1 ahead.
     const bool loader = t == 0;
     const int64_t row_codes = D * BITS / 8;
@@ -459,9 +471,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         VItem nxt = load_item(t);
 #pragma unroll 1
         for (int i = 0; i < kItersV; ++i) {
-          const int it = t + 128 * i, key = item_key<D>(it), blk = item_blk<D>(it);
+          const int it = t + kVThreads * i, key = item_key<D>(it), blk = item_blk<D>(it);
+          if (it >= kItems) break;
           const VItem cur = nxt;
-          if (i + 1 < kItersV) nxt = load_item(it + 128);
+          if (i + 1 < kItersV && it + kVThreads < kItems) nxt = load_item(it + kVThreads);
           uint32_t v[16];
           if (key < valid) {
             dequant32(cur.cv, cur.st, cur.zp, v);
@@ -483,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         const int64_t t0 = static_cast<int64_t>(j - Tc) * N;
         const int valid = static_cast<int>(cur_keys - t0 < N ? cur_keys - t0 : N);
         const uint4* src = reinterpret_cast<const uint4*>(p.V_cur) + (static_cast<int64_t>(bh) * p.Lcur + t0) * (D / 8);
-        copy_rows<D, N, kItersV, 128, false>(src, vt, valid, t);
+        copy_rows<D, N, kItersV, kVThreads, false>(src, vt, valid, t);
         fence_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_VH_FULL + sb));
