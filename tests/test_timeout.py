@@ -1,4 +1,4 @@
-"""The attention kernel's bounded waits: with the bound lowered to one cycle every wait that does
+"""The attention kernels' bounded waits: with the bound lowered to one cycle every wait that does
 not succeed at once gives up, the kernel drains its own copies and tensor-core operations, frees
 its tensor memory and returns; the device status word then reads QKV_ERR_TIMEOUT, the context
 stays usable, and the next call with the default bound passes parity on the same device.
@@ -38,3 +38,24 @@ def test_wait_bound_runs_out_then_next_call_passes(case):
     assert api.device_status(reset=True) == 0
     # same device, default bound: every row against the oracle
     check_full(w, correct=1)
+
+
+@pytest.mark.parametrize("Lq", [45, 1])
+def test_wait_bound_runs_out_per_channel_keys(Lq):
+    """The same for the tensor-core kernel of caches with per-channel key blocks (unsplit, and with
+    its cached keys split over CTAs for a one-row chunk)."""
+    from test_key_channel_parity import SMALL, build_chan_cache, check_every_row
+    w = SMALL["prefill_gqa"].with_(seed=317, Lq=Lq, Lcur=Lq, Lc=32 * 40 + 9 if Lq == 1 else 333)
+    assert api.device_status(reset=True) == 0
+    prev = api.set_wait_limit(1)
+    try:
+        x = make_inputs(w, device="cuda")
+        cache = build_chan_cache(w, x["K_src"], x["V_src"], 32)
+        api.corrected_attention(x["Q"], cache, x["K_cur"], x["V_cur"], correct=1, causal=w.causal,
+                                workspace="auto")
+        torch.cuda.synchronize()
+    finally:
+        api.set_wait_limit(prev)
+    assert api.device_status(reset=True) == api.QKV_ERR_TIMEOUT
+    assert api.device_status(reset=True) == 0
+    check_every_row(w, 32, 1)
