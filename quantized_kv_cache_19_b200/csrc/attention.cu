@@ -469,7 +469,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           return r;
         };
         VItem nxt = load_item(t);
-#pragma unroll 1
+        // Unrolled with one group (the long-video cache: 6.22 ms against 6.46), not with two (the
+        // chunked-prefill and video shapes gain nothing or lose 1%: instruction-cache pressure).
+#pragma unroll (NG == 1 ? kItersV : 1)
         for (int i = 0; i < kItersV; ++i) {
           const int it = t + kVThreads * i, key = item_key<D>(it), blk = item_blk<D>(it);
           if (it >= kItems) break;
