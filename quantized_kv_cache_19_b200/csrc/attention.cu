@@ -318,6 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     // ---------------------------------------------------------------- K operand tiles (warps 1-3)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = wg == 0 ? threadIdx.x - 32 : threadIdx.x - 512 + 96;   // 0 .. kKThreads - 1
+    // This thread's unpack items t, t + kKThreads, ...: one channel block, keys kKeyStep apart
+    // (item_key / item_blk of those indices), so their code and store addresses advance by
+    // constants.
+    constexpr int kKeyStep = kKThreads * 32 / D;
+    static_assert((kKThreads * 32) % D == 0 && kKeyStep % 8 == 0, "items of a thread share a block");
+    const int key0 = item_key<D>(t), blk0 = item_blk<D>(t);
+    uint32_t so[4];
+    chunk_offsets<N>(key0, blk0, so);
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* kt = smem + L.kt + sb * C::kTile;
@@ -332,19 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         // One item per iteration with the next item's codes already loaded (shared-memory loads
         // take ~170 cycles while the tensor core reads its operands), the loop itself not
         // unrolled: the code of all roles shares the instruction caches of each SM sub-partition.
-        auto load_codes = [&](int it) {
-          return *reinterpret_cast<const CodeVec*>(kcodes + item_key<D>(it) * (D * BITS / 8) +
-                                                   item_blk<D>(it) * (4 * BITS));
-        };
-        CodeVec cv_next = load_codes(t < kItems ? t : 0);
+        constexpr int kRowCodes = D * BITS / 8;
+        const uint8_t* src = kcodes + key0 * kRowCodes + blk0 * (4 * BITS);
+        uint8_t* row = kt + key0 * 128;
+        CodeVec cv_next = *reinterpret_cast<const CodeVec*>(src);
 #pragma unroll 1
-        for (int i = 0; i < kItersK; ++i) {
-          const int it = t + kKThreads * i;
-          if (it >= kItems) break;
+        for (int key = key0; key < N; key += kKeyStep, src += kKeyStep * kRowCodes, row += kKeyStep * 128) {
           const CodeVec cv = cv_next;
-          const int it_next = it + kKThreads;
-          if (it_next < kItems) cv_next = load_codes(it_next);
-          const int key = item_key<D>(it), blk = item_blk<D>(it);
+          if (key + kKeyStep < N) cv_next = *reinterpret_cast<const CodeVec*>(src + kKeyStep * kRowCodes);
           uint32_t v[16];
           if (key < valid) {
             unpack_codes32(cv, v);
@@ -352,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
-          store32<N>(kt, key, blk, v);
+          store_chunks(row, so, v);
         }
         // Per-key constants of the tile: scales a for the softmax (once it has read the previous
         // ones from this buffer) and the key extras of the S MMA.
@@ -372,21 +375,28 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
             else load_meta<false>(kmeta, key * NG + g, step, zp);
             const float sp = step > 0.f ? step : 1.f;     // a constant group has code 0 everywhere
             a = sp * p.scale_log2;
-            rho = zp / sp;
+            // rho = zp / step to within 2 ulp (reciprocal and multiply): its three bf16 parts keep
+            // ~24 bits, so the IEEE division's last ulp is not resolved anyway.
+            rho = __fdividef(zp, sp);
             sigma = step * p.inv_scale_log2;
             const float s2 = step * step;
             d4 = s2 * s2;                                 // fourth-order term (softmax, fp32)
           }
           const int ci = ((key >> 1) * C::NAH + (g >> 1)) * 4 + (g & 1) * 2 + (key & 1);
           kc[ci] = a;
-          kc[2 * (C::kKconst / 4) + ci] = d4;
-          __nv_bfloat16 rh, rm, rl, sh, sm, sl;
-          split3(rho, rh, rm, rl);
-          split3(sigma, sh, sm, sl);
+          if (kQuartic) kc[2 * (C::kKconst / 4) + ci] = d4;   // read by the softmax with correct = 2 only
+          // rho and sigma split together into three bf16 parts each (hi = RN(x), mid = RN(x - hi),
+          // lo = RN(x - hi - mid)), as pairs (rho part, sigma part)
+          const uint32_t hp = pack_bf16x2(rho, sigma);
+          const float2 r1 = make_float2(rho - bf16_lo(hp), sigma - bf16_hi(hp));
+          const uint32_t mp = pack_bf16x2(r1.x, r1.y);
+          const uint32_t lp = pack_bf16x2(r1.x - bf16_lo(mp), r1.y - bf16_hi(mp));
           // [rho_h, rho_m, rho_h, rho_l, rho_m, rho_h, sig_h, sig_m, sig_h, sig_l, sig_h, sig_m, 0, 0, 0, 0]
+          const uint32_t sig_hm = __byte_perm(hp, mp, 0x7632);
           store_extras(bx + sb * C::kBx + g * (N * 32), key,
-                       make_uint4(bf_pair(rh, rm), bf_pair(rh, rl), bf_pair(rm, rh), bf_pair(sh, sm)),
-                       make_uint4(bf_pair(sh, sl), bf_pair(sh, sm), 0u, 0u));
+                       make_uint4(__byte_perm(hp, mp, 0x5410), __byte_perm(hp, lp, 0x5410),
+                                  __byte_perm(mp, hp, 0x5410), sig_hm),
+                       make_uint4(__byte_perm(hp, lp, 0x7632), sig_hm, 0u, 0u));
         }
         fence_async_smem();
         __syncwarp();
@@ -421,6 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     // ---------------------------------------------------------------- V operand tiles
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = wg == 3 ? threadIdx.x - 384 : threadIdx.x - 32 * (16 + kKWarps - 3) + 128;  // 0 .. kVThreads - 1
+    // This thread's items t, t + kVThreads, ...: one channel block, keys kKeyStepV apart.
+    constexpr int kKeyStepV = kVThreads * 32 / D;
+    static_assert((kVThreads * 32) % D == 0 && kKeyStepV % 8 == 0, "items of a thread share a block");
+    const int vkey0 = item_key<D>(t), vblk0 = item_blk<D>(t);
+    uint32_t vso[4];
+    chunk_offsets<N>(vkey0, vblk0, vso);
     // Lane 0 of the first V warp also issues the bulk copies of packed tiles, kStages - 1 ahead.
     const bool loader = t == 0;
     const int64_t row_codes = D * BITS / 8;
@@ -460,23 +476,29 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         // (shared-memory loads are slow while the tensor core reads its operands); the loop itself
         // is not unrolled.
         struct VItem { CodeVec cv; float st, zp; };
-        auto load_item = [&](int it) {
+        constexpr int kRowCodes = D * BITS / 8;
+        const int mb2 = p.meta_f16 ? 4 : 8;                       // bytes of one (step, zero-point)
+        const uint8_t* csrc = vcodes + vkey0 * kRowCodes + vblk0 * (4 * BITS);
+        const uint8_t* msrc = vmeta + (vkey0 * NG + (vblk0 * 32) / C::G) * mb2;
+        const int mstep = kKeyStepV * NG * mb2;
+        auto load_item = [&](const uint8_t* cp, const uint8_t* mp) {
           VItem r;
-          const int key = item_key<D>(it), blk = item_blk<D>(it), g = (blk * 32) / C::G;
-          r.cv = *reinterpret_cast<const CodeVec*>(vcodes + key * (D * BITS / 8) + blk * (4 * BITS));
-          if (p.meta_f16) load_meta<true>(vmeta, key * NG + g, r.st, r.zp);
-          else load_meta<false>(vmeta, key * NG + g, r.st, r.zp);
+          r.cv = *reinterpret_cast<const CodeVec*>(cp);
+          if (p.meta_f16) load_meta<true>(mp, 0, r.st, r.zp);
+          else load_meta<false>(mp, 0, r.st, r.zp);
           return r;
         };
-        VItem nxt = load_item(t);
+        VItem nxt = load_item(csrc, msrc);
+        uint8_t* vrow = vt + vkey0 * 128;
         // Unrolled with one group (the long-video cache: 6.22 ms against 6.46), not with two (the
         // chunked-prefill and video shapes gain nothing or lose 1%: instruction-cache pressure).
 #pragma unroll (NG == 1 ? kItersV : 1)
         for (int i = 0; i < kItersV; ++i) {
-          const int it = t + kVThreads * i, key = item_key<D>(it), blk = item_blk<D>(it);
-          if (it >= kItems) break;
+          const int key = vkey0 + kKeyStepV * i;
+          if (key >= N) break;
           const VItem cur = nxt;
-          if (i + 1 < kItersV && it + kVThreads < kItems) nxt = load_item(it + kVThreads);
+          if (i + 1 < kItersV && key + kKeyStepV < N)
+            nxt = load_item(csrc + (i + 1) * (kKeyStepV * kRowCodes), msrc + (i + 1) * mstep);
           uint32_t v[16];
           if (key < valid) {
             dequant32(cur.cv, cur.st, cur.zp, v);
@@ -484,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
-          store32<N>(vt, key, blk, v);
+          store_chunks(vrow + i * (kKeyStepV * 128), vso, v);
         }
         fence_async_smem();
         __syncwarp();

@@ -140,6 +140,24 @@ __device__ __forceinline__ void store32(uint8_t* tile, int key, int blk, const u
   }
 }
 
+// The 16-byte chunks of one (key, 32-channel block) item in a [d/64][N][64] tile with the 128-byte
+// swizzle, as byte offsets from the start of the key's row (tile + key * 128; store32 writes the
+// same addresses). They depend on the key only through key % 8, so a thread whose items lie a
+// multiple of 8 keys apart keeps them for all its items and advances one row pointer.
+template <int N>
+__device__ __forceinline__ void chunk_offsets(int key, int blk, uint32_t (&o)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = blk * 4 + i;
+    o[i] = (c >> 3) * (N * 128) + (((c & 7) ^ (key & 7)) << 4);
+  }
+}
+__device__ __forceinline__ void store_chunks(uint8_t* row, const uint32_t (&o)[4], const uint32_t (&v)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint4*>(row + o[i]) = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
 template <bool F16>
 __device__ __forceinline__ void load_meta(const uint8_t* meta, int idx, float& step, float& zp) {
   if (F16) {
