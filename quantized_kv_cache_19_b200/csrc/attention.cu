@@ -326,6 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     const int key0 = item_key<D>(t), blk0 = item_blk<D>(t);
     uint32_t so[4];
     chunk_offsets<N>(key0, blk0, so);
+    // Per-key-constant items t, t + kKThreads, ...: (key, group) = (e / NG, e % NG), one group,
+    // keys kKeyStepC apart; the scale index and the extras row advance by constants.
+    constexpr int kKeyStepC = kKThreads / NG;
+    static_assert(kKThreads % NG == 0 && kKeyStepC % 8 == 0, "constant items of a thread share a group");
+    const int gc = t % NG, keyc0 = t / NG;
+    const int ci0 = ((keyc0 >> 1) * C::NAH + (gc >> 1)) * 4 + (gc & 1) * 2 + (keyc0 & 1);
+    const int xo0 = gc * (N * 32) + (keyc0 >> 3) * 256 + (keyc0 & 7) * 16;   // store_extras layout
     for (int j = 0; j < T; ++j) {
       const int sb = j & 1, n = j >> 1;
       uint8_t* kt = smem + L.kt + sb * C::kTile;
@@ -365,14 +372,13 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         constexpr int kItersC = (N * NG + kKThreads - 1) / kKThreads;
 #pragma unroll 1
         for (int i = 0; i < kItersC; ++i) {
-          const int e = t + kKThreads * i;
-          if (e >= N * NG) break;
-          const int key = e / NG, g = e % NG;
+          const int key = keyc0 + kKeyStepC * i;
+          if (key >= N) break;
           float a = 0.f, rho = 0.f, sigma = 0.f, d4 = 0.f;
           if (key < valid) {
             float step, zp;
-            if (p.meta_f16) load_meta<true>(kmeta, key * NG + g, step, zp);
-            else load_meta<false>(kmeta, key * NG + g, step, zp);
+            if (p.meta_f16) load_meta<true>(kmeta, t + kKThreads * i, step, zp);
+            else load_meta<false>(kmeta, t + kKThreads * i, step, zp);
             const float sp = step > 0.f ? step : 1.f;     // a constant group has code 0 everywhere
             a = sp * p.scale_log2;
             // rho = zp / step to within 2 ulp (reciprocal and multiply): its three bf16 parts keep
@@ -382,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
             const float s2 = step * step;
             d4 = s2 * s2;                                 // fourth-order term (softmax, fp32)
           }
-          const int ci = ((key >> 1) * C::NAH + (g >> 1)) * 4 + (g & 1) * 2 + (key & 1);
+          const int ci = ci0 + i * (kKeyStepC / 2) * C::NAH * 4;
           kc[ci] = a;
           if (kQuartic) kc[2 * (C::kKconst / 4) + ci] = d4;   // read by the softmax with correct = 2 only
           // rho and sigma split together into three bf16 parts each (hi = RN(x), mid = RN(x - hi),
@@ -393,10 +399,11 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
           const uint32_t lp = pack_bf16x2(r1.x - bf16_lo(mp), r1.y - bf16_hi(mp));
           // [rho_h, rho_m, rho_h, rho_l, rho_m, rho_h, sig_h, sig_m, sig_h, sig_l, sig_h, sig_m, 0, 0, 0, 0]
           const uint32_t sig_hm = __byte_perm(hp, mp, 0x7632);
-          store_extras(bx + sb * C::kBx + g * (N * 32), key,
-                       make_uint4(__byte_perm(hp, mp, 0x5410), __byte_perm(hp, lp, 0x5410),
-                                  __byte_perm(mp, hp, 0x5410), sig_hm),
-                       make_uint4(__byte_perm(hp, lp, 0x7632), sig_hm, 0u, 0u));
+          // the extras row of (key, group): [row / 8][2 halves][row % 8][8] (store_extras' layout)
+          uint8_t* xrow = bx + sb * C::kBx + xo0 + i * ((kKeyStepC / 8) * 256);
+          *reinterpret_cast<uint4*>(xrow) = make_uint4(__byte_perm(hp, mp, 0x5410), __byte_perm(hp, lp, 0x5410),
+                                                       __byte_perm(mp, hp, 0x5410), sig_hm);
+          *reinterpret_cast<uint4*>(xrow + 128) = make_uint4(__byte_perm(hp, lp, 0x7632), sig_hm, 0u, 0u);
         }
         fence_async_smem();
         __syncwarp();

@@ -440,6 +440,11 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
     const int t = threadIdx.x - 384;
     constexpr int kItems = kN * (D / 32);
     constexpr int kItersV = kItems / 128;
+    // This thread's items t, t + 128, ...: one channel block, keys 32 apart.
+    constexpr int kKeyStepV = 128 * 32 / D;
+    const int vkey0 = item_key<D>(t), vblk0 = item_blk<D>(t);
+    uint32_t vso[4];
+    chunk_offsets<kN>(vkey0, vblk0, vso);
     const bool loader = t == 0;
     const int64_t row_codes = D * BITS / 8;
     const int64_t vrow_meta = static_cast<int64_t>(NGV) * 2 * (p.meta_f16 ? 2 : 4);
@@ -477,22 +482,24 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
         const uint8_t* vmeta = smem + L.pk + s * L.stage + 2 * C::kCodes + L.kmeta;
         if (!waitw(B_PK_FULL + s, k & 1)) break;
         using CodeVec = typename CodeVecT<BITS>::type;
+        const uint8_t* csrc = vcodes + vkey0 * row_codes + vblk0 * (4 * BITS);
+        const int mb2 = p.meta_f16 ? 4 : 8;
+        const uint8_t* msrc = vmeta + (vkey0 * NGV + (vblk0 * 32) / C::GV) * mb2;
 #pragma unroll 1
         for (int i = 0; i < kItersV; ++i) {
-          const int it = t + 128 * i, key = item_key<D>(it), blk = item_blk<D>(it);
+          const int key = vkey0 + kKeyStepV * i;
           uint32_t v[16];
           if (key < valid) {
-            const int g = (blk * 32) / C::GV;
-            const CodeVec cv = *reinterpret_cast<const CodeVec*>(vcodes + key * row_codes + blk * (4 * BITS));
+            const CodeVec cv = *reinterpret_cast<const CodeVec*>(csrc + i * (kKeyStepV * row_codes));
             float st, zp;
-            if (p.meta_f16) load_meta<true>(vmeta, key * NGV + g, st, zp);
-            else load_meta<false>(vmeta, key * NGV + g, st, zp);
+            if (p.meta_f16) load_meta<true>(msrc + i * (kKeyStepV * NGV * mb2), 0, st, zp);
+            else load_meta<false>(msrc + i * (kKeyStepV * NGV * mb2), 0, st, zp);
             dequant32(cv, st, zp, v);
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = 0u;
           }
-          store32<kN>(vt, key, blk, v);
+          store_chunks(vt + (vkey0 + kKeyStepV * i) * 128, vso, v);
         }
         fence_async_smem();
         __syncwarp();
