@@ -649,6 +649,11 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       // s = sum_g a_g * S_g: per-key group scales for cached tiles, the score scale for current ones.
       const float4* ka = kconst + kb * (C::kKconst / 16);
       const float4* kd4 = kconst + (2 + kb) * (C::kKconst / 16);
+      // Scores are formed relative to the maximum in use so far (m_prev, 0 before the first key):
+      // the exponentials then need no subtraction unless the maximum moves, which lazy rescaling
+      // makes rare.
+      const float m_prev = m_run == -INFINITY ? 0.f : m_run;
+      const float2 mprev2 = make_float2(-m_prev, -m_prev);
 #pragma unroll
       for (int c0 = 0; c0 < NH; c0 += kCK) {
         // (After a failed wait these loads read whatever the accumulators hold; the values are
@@ -660,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
 #pragma unroll
         for (int q = 0; q < kCK / 2; ++q) {
           const int pq = (kbase_h + c0) / 2 + q;
-          float2 acc = make_float2(0.f, 0.f);
+          float2 acc = mprev2;                    // scores relative to the running maximum
 #pragma unroll
           for (int ah = 0; ah < C::NAH; ++ah) {
             const float4 a = ka[pq * C::NAH + ah];
@@ -705,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       const float m_half = fmax3(fmaxf(m0, m1), m2, m3);
       xmax[((j & 1) * 2 + half) * kBM + row] = m_half;
       if (named_sync_or(1, 256, !ok)) { ok = false; break; }
-      const float m_tile = fmaxf(m_half, xmax[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
+      const float m_tile = fmaxf(m_half, xmax[((j & 1) * 2 + (half ^ 1)) * kBM + row]) + m_prev;
       // Lazy rescaling: keep the old max unless the new one exceeds it by the threshold.
       const bool need = (m_tile > m_run + kRescaleThreshold) ||
                         (m_run == -INFINITY && m_tile > -INFINITY);
@@ -716,8 +721,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         m_run = m_tile;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const bool any_need = __any_sync(0xffffffffu, need);
       // O is rescaled only after the previous P.V has finished (rare with lazy rescaling).
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (j > 0 && any_need) {
         if (!warp_wait(bar(B_PV_DONE + (j - 1) % C::kPB), ((j - 1) / C::kPB) & 1, abort_flag, p.status, p.wait_limit)) { ok = false; continue; }
         tc_fence_after();
         const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
@@ -741,12 +747,16 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         if (!warp_wait(bar(B_PV_DONE + pb), ((j - C::kPB) / C::kPB) & 1, abort_flag, p.status, p.wait_limit)) { ok = false; continue; }
         tc_fence_after();
       }
-      const float2 mneg = make_float2(-m_use, -m_use);
+      if (any_need) {                           // the maximum moved: scores relative to the new one
+        const float2 d2 = make_float2(m_prev - m_use, m_prev - m_use);
+#pragma unroll
+        for (int k = 0; k < NH / 2; ++k) s2[k] = __fadd2_rn(s2[k], d2);
+      }
       float2 psum = make_float2(0.f, 0.f);
       uint32_t pk[NH / 2];
 #pragma unroll
       for (int k = 0; k < NH / 2; ++k) {
-        const float2 e = __fadd2_rn(s2[k], mneg);
+        const float2 e = s2[k];
         const float2 pp = make_float2(ex2(e.x), ex2(e.y));
         psum = __fadd2_rn(psum, pp);
         pk[k] = pack_bf16x2(pp.x, pp.y);
