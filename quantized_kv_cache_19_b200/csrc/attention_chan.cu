@@ -611,6 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
         valid = static_cast<int>(lim < 0 ? 0 : (lim < kN ? lim : kN));
       }
       // The correction of each block of the tile (log2 units), for cached tiles.
+      // Scores relative to the maximum in use so far (0 before the first key), as in the
+      // per-token kernel: no subtraction in the exponentials unless the maximum moves.
+      const float m_prev = m_run == -INFINITY ? 0.f : m_run;
       float corr[4] = {0.f, 0.f, 0.f, 0.f};
       if (cached && p.correct) {
         uint32_t cr[8];
@@ -632,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
         // 32 keys of one block (T is a multiple of 32).
         const int bk = (kbase_h + cc) / T;
         const float cb = bk == 0 ? corr[0] : (bk == 1 ? corr[1] : (bk == 2 ? corr[2] : corr[3]));
-        const float2 nc = make_float2(-cb, -cb);
+        const float2 nc = make_float2(-cb - m_prev, -cb - m_prev);
 #pragma unroll
         for (int q = 0; q < 16; ++q)
           s2[cc / 2 + q] = __ffma2_rn(scale2, make_float2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1])), nc);
@@ -658,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
       const float m_half = fmax3(fmaxf(m0, m1), m2, m3);
       xmax[((j & 1) * 2 + half) * kBM + row] = m_half;
       if (named_sync_or(1, 256, !ok)) { ok = false; break; }
-      const float m_tile = fmaxf(m_half, xmax[((j & 1) * 2 + (half ^ 1)) * kBM + row]);
+      const float m_tile = fmaxf(m_half, xmax[((j & 1) * 2 + (half ^ 1)) * kBM + row]) + m_prev;
       const bool need = (m_tile > m_run + kRescaleThreshold) || (m_run == -INFINITY && m_tile > -INFINITY);
       float factor = 1.f;
       if (need) {
@@ -667,11 +670,12 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
         m_run = m_tile;
       }
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const bool any_need = __any_sync(0xffffffffu, need);
       // O is rescaled after the previous P.V has finished; P is rewritten after it too (one buffer).
       if (j > 0) {
         if (!waitw(B_PV_DONE, (j - 1) & 1)) { ok = false; continue; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        if (any_need) {
           const uint32_t tm_o = tmem + lane_off + kColO + half * (D / 2);
           const float2 f2 = make_float2(factor, factor);
 #pragma unroll 1
@@ -689,12 +693,16 @@ __global__ void __launch_bounds__(kThreads, 1) chan_attention_kernel(const AttnP
           }
         }
       }
-      const float2 mneg = make_float2(-m_use, -m_use);
+      if (any_need) {
+        const float2 d2 = make_float2(m_prev - m_use, m_prev - m_use);
+#pragma unroll
+        for (int k = 0; k < NH / 2; ++k) s2[k] = __fadd2_rn(s2[k], d2);
+      }
       float2 psum = make_float2(0.f, 0.f);
       uint32_t pk[NH / 2];
 #pragma unroll
       for (int k = 0; k < NH / 2; ++k) {
-        const float2 e = __fadd2_rn(s2[k], mneg);
+        const float2 e = s2[k];
         const float2 pp = make_float2(ex2(e.x), ex2(e.y));
         psum = __fadd2_rn(psum, pp);
         pk[k] = pack_bf16x2(pp.x, pp.y);
