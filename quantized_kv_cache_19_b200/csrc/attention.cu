@@ -645,6 +645,10 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
         }
         valid = static_cast<int>(lim < 0 ? 0 : (lim < N ? lim : N));
       }
+      // The first group's first chunk of S is loaded from tensor memory while this warp waits for
+      // the tile's per-key scales.
+      uint32_t r[C::NA][kCK];
+      tmem_ld<kCK>(tm_s, r[0]);
       if (ok && !warp_wait(bar(B_KC_FULL + kb), (j >> 1) & 1, abort_flag, p.status, p.wait_limit)) ok = false;
       // s = sum_g a_g * S_g: per-key group scales for cached tiles, the score scale for current ones.
       const float4* ka = kconst + kb * (C::kKconst / 16);
@@ -658,9 +662,9 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
       for (int c0 = 0; c0 < NH; c0 += kCK) {
         // (After a failed wait these loads read whatever the accumulators hold; the values are
         // dropped at the exchange below, where the warps leave the loop.)
-        uint32_t r[C::NA][kCK];
 #pragma unroll
-        for (int a = 0; a < C::NA; ++a) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
+        for (int a = 0; a < C::NA; ++a)
+          if (c0 > 0 || a > 0) tmem_ld<kCK>(tm_s + a * N + c0, r[a]);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < kCK / 2; ++q) {
