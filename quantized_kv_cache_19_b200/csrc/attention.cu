@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1) corrected_attention_kernel(const 
     }
     __syncwarp();
   } else if (wg == 0 || (wg == 4 && warp < 16 + kKWarps - 3)) {
-    // ---------------------------------------------------------------- K operand tiles (warps 1-3)
+    // ---------------------------------------------------------------- K operand tiles (warps 1-3, 16..)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegProducer));
     const int t = wg == 0 ? threadIdx.x - 32 : threadIdx.x - 512 + 96;   // 0 .. kKThreads - 1
     // This thread's unpack items t, t + kKThreads, ...: one channel block, keys kKeyStep apart
